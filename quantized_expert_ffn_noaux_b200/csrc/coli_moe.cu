@@ -1,0 +1,726 @@
+// coli_moe.cu -- host side of the C ABI declared in include/coli_moe.h.
+//
+// Validates arguments, owns the per-handle device workspace, and enqueues the
+// kernels of quant.cuh, route.cuh and expert.cuh on the caller's stream.
+// No call synchronises the host except coli_moe_forward_host.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "coli_moe.h"
+#include "common.cuh"
+#include "expert.cuh"
+#include "quant.cuh"
+#include "route.cuh"
+
+using namespace coli;
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<uint64_t> g_launches{0};
+
+coli_status fail(coli_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+coli_status cuda_fail(cudaError_t e, const char *what) {
+    cudaGetLastError();  // clear the sticky-free error state of the runtime
+    return fail(e == cudaErrorMemoryAllocation ? COLI_ENOMEM : COLI_ECUDA, "%s: %s", what,
+                cudaGetErrorString(e));
+}
+
+#define COLI_CUDA(call, what)                          \
+    do {                                               \
+        cudaError_t e_ = (call);                       \
+        if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+    } while (0)
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+    return n > 0 ? n : 148;
+}
+
+constexpr int MAX_SMEM = 227 * 1024;
+constexpr int SMALL_T = 8;  // the few-token down+combine path handles T <= SMALL_T
+
+// Vectors per lane template choice for a row of V uint4 vectors.
+int pick_vpl(int V) {
+    int need = (V + 31) / 32;
+    if (need <= 1) return 1;
+    if (need <= 2) return 2;
+    if (need <= 4) return 4;
+    if (need <= 6) return 6;
+    if (need <= 12) return 12;
+    return 0;  // generic loop
+}
+
+struct KernelTimer {
+    const char *name;
+    cudaEvent_t a, b;
+};
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+struct coli_moe {
+    coli_moe_config cfg;
+    const float *router_w = nullptr, *bias = nullptr;
+    int device = 0, nsm = 148;
+    void *ws_base = nullptr;
+    size_t ws_bytes = 0;
+    RouteWs rw{};
+    ExpertDev *experts_dev = nullptr;
+    int8_t *xq = nullptr;
+    float *xd = nullptr;
+    int8_t *hq = nullptr;
+    float *hd = nullptr;
+    float *e_pairs = nullptr;  // only when max_tokens > SMALL_T
+    float *x_in = nullptr, *y_out = nullptr;
+    int last_T = 0;
+    std::map<const void *, int> occ_cache;  // kernel -> CTAs per SM (attributes already set)
+    // profiling
+    bool profiling = false;
+    std::vector<KernelTimer> pending;
+    std::vector<cudaEvent_t> event_pool;
+};
+
+namespace {
+
+struct Layout {
+    size_t total = 0;
+    size_t add(size_t bytes) {
+        size_t off = (total + 255) & ~(size_t)255;
+        total = off + bytes;
+        return off;
+    }
+};
+
+struct WsOffsets {
+    size_t s, c, idx, w, bitmap, prefix, counter, n_active, active, off, act_of, pair_tok,
+        pair_slot, tok_pair, xq, xd, hq, hd, e_pairs, x_in, y_out, experts;
+    size_t total;
+};
+
+bool cfg_valid(const coli_moe_config *c, std::string *why) {
+    auto bad = [&](const char *m) {
+        if (why) *why = m;
+        return false;
+    };
+    if (!c) return bad("cfg is NULL");
+    if (c->wfmt != 8 && c->wfmt != 4 && c->wfmt != 2) return bad("wfmt must be 8, 4 or 2");
+    const int q = c->wfmt == 2 ? 64 : 32;
+    if (c->hidden <= 0 || c->hidden % q || c->hidden > 16384)
+        return bad("hidden must be a positive multiple of 32 (64 for int2), <= 16384");
+    if (c->inter <= 0 || c->inter % q || c->inter > 16384)
+        return bad("inter must be a positive multiple of 32 (64 for int2), <= 16384");
+    if (c->n_routed < 1 || c->n_routed > 1024) return bad("n_routed must be in [1, 1024]");
+    if (c->n_shared < 0 || c->n_shared > 4) return bad("n_shared must be in [0, 4]");
+    if (c->n_group < 1 || c->n_routed % c->n_group) return bad("n_group must divide n_routed");
+    if (c->topk_group < 1 || c->topk_group > c->n_group) return bad("topk_group must be in [1, n_group]");
+    const int cand = c->topk_group * (c->n_routed / c->n_group);
+    if (c->top_k < 1 || c->top_k > 32 || c->top_k > cand)
+        return bad("top_k must be in [1, min(32, topk_group * n_routed / n_group)]");
+    if (!(c->routed_scaling_factor == c->routed_scaling_factor)) return bad("routed_scaling_factor is NaN");
+    if (c->max_tokens < 1 || c->max_tokens > (1 << 20)) return bad("max_tokens must be in [1, 2^20]");
+    return true;
+}
+
+WsOffsets layout_of(const coli_moe_config &c) {
+    Layout L;
+    WsOffsets o{};
+    const size_t T = c.max_tokens, E = c.n_routed, S = c.n_shared, k = c.top_k;
+    const size_t H = c.hidden, I = c.inter;
+    const size_t P = T * (k + S);
+    const size_t wstride = (T + 31) / 32;
+    o.s = L.add(T * E * 8);
+    o.c = L.add(T * E * 8);
+    o.idx = L.add(T * k * 4);
+    o.w = L.add(T * k * 4);
+    o.bitmap = L.add(E * wstride * 4);
+    o.prefix = L.add(E * wstride * 4);
+    o.counter = L.add(4);
+    o.n_active = L.add(4);
+    o.active = L.add((E + S) * 4);
+    o.off = L.add((E + S + 1) * 4);
+    o.act_of = L.add((E + S) * 4);
+    o.pair_tok = L.add(P * 4);
+    o.pair_slot = L.add(P * 4);
+    o.tok_pair = L.add(P * 4);
+    o.xq = L.add(T * H);
+    o.xd = L.add(T * (H / 32) * 4);
+    o.hq = L.add(P * I);
+    o.hd = L.add(P * (I / 32) * 4);
+    o.e_pairs = (T > (size_t)SMALL_T) ? L.add(P * H * 4) : 0;
+    o.x_in = L.add(T * H * 4);
+    o.y_out = L.add(T * H * 4);
+    o.experts = L.add((E + S) * sizeof(ExpertDev));
+    o.total = L.total;
+    return o;
+}
+
+// --- launch helpers --------------------------------------------------------
+cudaEvent_t pool_event(coli_moe *m) {
+    if (!m->event_pool.empty()) {
+        cudaEvent_t e = m->event_pool.back();
+        m->event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+struct Launch {
+    coli_moe *m;
+    cudaStream_t s;
+    const char *name;
+    cudaEvent_t a = nullptr;
+    Launch(coli_moe *m_, cudaStream_t s_, const char *n) : m(m_), s(s_), name(n) {
+        if (m && m->profiling) {
+            a = pool_event(m);
+            if (a) cudaEventRecord(a, s);
+        }
+    }
+    coli_status done() {
+        cudaError_t e = cudaGetLastError();
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        if (m && m->profiling && a) {
+            cudaEvent_t b = pool_event(m);
+            if (b) {
+                cudaEventRecord(b, s);
+                m->pending.push_back({name, a, b});
+            }
+        }
+        if (e != cudaSuccess) return cuda_fail(e, name);
+        return COLI_OK;
+    }
+};
+
+// Set the kernel's shared-memory limit and return its CTAs per SM, once per
+// (handle, kernel); later calls (e.g. during CUDA graph capture) only read the cache.
+template <typename K>
+coli_status prepare(coli_moe *m, K kernel, int threads, size_t smem, int *occ);
+
+template <typename K>
+coli_status allow_smem(K kernel, size_t bytes) {
+    if (bytes > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)bytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    }
+    return COLI_OK;
+}
+
+template <typename K>
+int occupancy(K kernel, int threads, size_t smem) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess)
+        return 1;
+    return n > 0 ? n : 1;
+}
+
+template <typename K>
+coli_status prepare(coli_moe *m, K kernel, int threads, size_t smem, int *occ) {
+    // the key includes the shared-memory size: the few-token down kernel's
+    // footprint depends on T
+    const void *key = (const void *)((uintptr_t)(const void *)kernel ^ ((uintptr_t)smem << 40));
+    auto it = m->occ_cache.find(key);
+    if (it != m->occ_cache.end()) {
+        *occ = it->second;
+        return COLI_OK;
+    }
+    coli_status st = allow_smem(kernel, smem);
+    if (st != COLI_OK) return st;
+    const int o = occupancy(kernel, threads, smem);
+    m->occ_cache[key] = o;
+    *occ = o;
+    return COLI_OK;
+}
+
+// --- kernel dispatch by (BITS, VPL) ------------------------------------------
+template <int BITS, int VPL>
+coli_status launch_gateup_t(coli_moe *m, int max_items, cudaStream_t s) {
+    const auto &c = m->cfg;
+    auto kern = k_gateup<BITS, VPL>;
+    size_t smem = stage_bytes(GROUP_NT, c.hidden) + 2 * ROWS_PER_ITEM * GROUP_NT * 4;
+    int occ = 1;
+    coli_status st = prepare(m, kern, 256, smem, &occ);
+    if (st != COLI_OK) return st;
+    int grid = std::min(max_items, m->nsm * occ);
+    grid = std::max(grid, 1);
+    Launch L(m, s, "gateup_swiglu_q8");
+    kern<<<grid, 256, smem, s>>>(m->rw, m->experts_dev, m->xq, m->xd, c.hidden, c.inter, m->hq,
+                                 m->hd);
+    return L.done();
+}
+
+template <int BITS>
+coli_status launch_gateup(coli_moe *m, int max_items, cudaStream_t s) {
+    switch (pick_vpl(m->cfg.hidden * BITS / 128)) {
+        case 1: return launch_gateup_t<BITS, 1>(m, max_items, s);
+        case 2: return launch_gateup_t<BITS, 2>(m, max_items, s);
+        case 4: return launch_gateup_t<BITS, 4>(m, max_items, s);
+        case 6: return launch_gateup_t<BITS, 6>(m, max_items, s);
+        case 12: return launch_gateup_t<BITS, 12>(m, max_items, s);
+        default: return launch_gateup_t<BITS, 0>(m, max_items, s);
+    }
+}
+
+template <int BITS, int VPL>
+coli_status launch_down_small_t(coli_moe *m, int T, float *out, cudaStream_t s) {
+    const auto &c = m->cfg;
+    auto kern = k_down_combine<BITS, VPL>;
+    const size_t P = (size_t)T * (c.top_k + c.n_shared);
+    size_t smem = stage_bytes((int)P, c.inter) + (size_t)GROUP_WARPS * P * DOWN_ROWS * 8;
+    int occ = 1;
+    coli_status st = prepare(m, kern, 256, smem, &occ);
+    if (st != COLI_OK) return st;
+    const int groups = c.hidden / DOWN_ROWS;
+    int grid = std::min((groups + GROUP_WARPS - 1) / GROUP_WARPS, m->nsm * occ);
+    grid = std::max(grid, 1);
+    Launch L(m, s, "down_combine");
+    kern<<<grid, 256, smem, s>>>(m->rw, m->experts_dev, m->hq, m->hd, T, c.hidden, c.inter,
+                                 c.top_k, c.n_shared, out);
+    return L.done();
+}
+
+template <int BITS>
+coli_status launch_down_small(coli_moe *m, int T, float *out, cudaStream_t s) {
+    switch (pick_vpl(m->cfg.inter * BITS / 128)) {
+        case 1: return launch_down_small_t<BITS, 1>(m, T, out, s);
+        case 2: return launch_down_small_t<BITS, 2>(m, T, out, s);
+        case 4: return launch_down_small_t<BITS, 4>(m, T, out, s);
+        case 6: return launch_down_small_t<BITS, 6>(m, T, out, s);
+        case 12: return launch_down_small_t<BITS, 12>(m, T, out, s);
+        default: return launch_down_small_t<BITS, 0>(m, T, out, s);
+    }
+}
+
+template <int BITS, int VPL>
+coli_status launch_down_grouped_t(coli_moe *m, int max_items, cudaStream_t s) {
+    const auto &c = m->cfg;
+    auto kern = k_down_grouped<BITS, VPL>;
+    size_t smem = stage_bytes(GROUP_NT, c.inter);
+    int occ = 1;
+    coli_status st = prepare(m, kern, 256, smem, &occ);
+    if (st != COLI_OK) return st;
+    int grid = std::max(1, std::min(max_items, m->nsm * occ));
+    Launch L(m, s, "down_grouped");
+    kern<<<grid, 256, smem, s>>>(m->rw, m->experts_dev, m->hq, m->hd, c.hidden, c.inter,
+                                 m->e_pairs);
+    return L.done();
+}
+
+template <int BITS>
+coli_status launch_down_grouped(coli_moe *m, int max_items, cudaStream_t s) {
+    switch (pick_vpl(m->cfg.inter * BITS / 128)) {
+        case 1: return launch_down_grouped_t<BITS, 1>(m, max_items, s);
+        case 2: return launch_down_grouped_t<BITS, 2>(m, max_items, s);
+        case 4: return launch_down_grouped_t<BITS, 4>(m, max_items, s);
+        case 6: return launch_down_grouped_t<BITS, 6>(m, max_items, s);
+        case 12: return launch_down_grouped_t<BITS, 12>(m, max_items, s);
+        default: return launch_down_grouped_t<BITS, 0>(m, max_items, s);
+    }
+}
+
+size_t select_smem(const coli_moe_config &c) {
+    return (size_t)c.n_routed * 8 + (size_t)c.n_group * 12 + (size_t)c.top_k * 4 + 16;
+}
+
+coli_status launch_route(coli_moe *m, const float *x, int T, int32_t *idx, float *w,
+                         int do_union, cudaStream_t s) {
+    const auto &c = m->cfg;
+    const int E = c.n_routed, H = c.hidden;
+    {
+        Launch L(m, s, "router_logits");
+        if (T <= 8) {
+            const int grid = (E + 7) / 8;
+            switch (T) {
+                case 1: k_route_logits_small<1><<<grid, 256, 0, s>>>(x, T, H, m->router_w, m->bias, E, m->rw.s, m->rw.c); break;
+                case 2: k_route_logits_small<2><<<grid, 256, 0, s>>>(x, T, H, m->router_w, m->bias, E, m->rw.s, m->rw.c); break;
+                case 3:
+                case 4: k_route_logits_small<4><<<grid, 256, 0, s>>>(x, T, H, m->router_w, m->bias, E, m->rw.s, m->rw.c); break;
+                default: k_route_logits_small<8><<<grid, 256, 0, s>>>(x, T, H, m->router_w, m->bias, E, m->rw.s, m->rw.c); break;
+            }
+        } else {
+            dim3 grid((T + 63) / 64, (E + 63) / 64);
+            k_route_logits_tiled<<<grid, 256, 0, s>>>(x, T, H, m->router_w, m->bias, E, m->rw.s,
+                                                      m->rw.c);
+        }
+        coli_status st = L.done();
+        if (st != COLI_OK) return st;
+    }
+    {
+        size_t smem = select_smem(c);
+        int occ = 1;
+        coli_status st = m ? prepare(m, k_route_select, 256, smem, &occ)
+                           : allow_smem(k_route_select, smem);
+        if (st != COLI_OK) return st;
+        Launch L(m, s, "router_select");
+        k_route_select<<<T, 256, smem, s>>>(m->rw, T, E, c.n_shared, c.n_group, c.topk_group,
+                                            c.top_k, c.routed_scaling_factor, idx, w, do_union);
+        return L.done();
+    }
+}
+
+coli_status quant_q8_launch(coli_moe *m, const float *x, int64_t rows, int64_t len, int8_t *q,
+                            float *d, cudaStream_t s) {
+    const int64_t nblocks = rows * (len / COLI_QBLK);
+    if (nblocks == 0) return COLI_OK;
+    const int64_t warps = 8;
+    int64_t grid = std::min<int64_t>((nblocks + warps - 1) / warps, (int64_t)sm_count() * 16);
+    Launch L(m, s, "quant_q8");
+    k_quant_q8<<<(unsigned)grid, 256, 0, s>>>(x, nblocks, q, d);
+    return L.done();
+}
+
+coli_status check_handle(coli_moe *m) {
+    if (!m) return fail(COLI_EINVAL, "handle is NULL");
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != m->device)
+        return fail(COLI_EINVAL, "current device %d is not the handle's device %d", dev, m->device);
+    return COLI_OK;
+}
+
+coli_status forward_impl(coli_moe *m, const float *x, int T, float *out, cudaStream_t s) {
+    const auto &c = m->cfg;
+    coli_status st;
+    st = quant_q8_launch(m, x, T, c.hidden, m->xq, m->xd, s);
+    if (st != COLI_OK) return st;
+    st = launch_route(m, x, T, m->rw.idx, m->rw.w, 1, s);
+    if (st != COLI_OK) return st;
+    const int max_active = std::min(c.n_routed, T * c.top_k) + c.n_shared;
+    const int gu_items = max_active * (c.inter / ROWS_PER_ITEM);
+    switch (c.wfmt) {
+        case 8: st = launch_gateup<8>(m, gu_items, s); break;
+        case 4: st = launch_gateup<4>(m, gu_items, s); break;
+        default: st = launch_gateup<2>(m, gu_items, s); break;
+    }
+    if (st != COLI_OK) return st;
+    const size_t P = (size_t)T * (c.top_k + c.n_shared);
+    const size_t small_smem = stage_bytes((int)P, c.inter) + (size_t)GROUP_WARPS * P * DOWN_ROWS * 8;
+    if (T <= SMALL_T && small_smem <= (size_t)MAX_SMEM) {
+        switch (c.wfmt) {
+            case 8: st = launch_down_small<8>(m, T, out, s); break;
+            case 4: st = launch_down_small<4>(m, T, out, s); break;
+            default: st = launch_down_small<2>(m, T, out, s); break;
+        }
+        if (st != COLI_OK) return st;
+    } else {
+        if (!m->e_pairs) return fail(COLI_EUNSUPPORTED, "T=%d needs the grouped down path", T);
+        const int dn_items = max_active * (c.hidden / ROWS_PER_ITEM);
+        switch (c.wfmt) {
+            case 8: st = launch_down_grouped<8>(m, dn_items, s); break;
+            case 4: st = launch_down_grouped<4>(m, dn_items, s); break;
+            default: st = launch_down_grouped<2>(m, dn_items, s); break;
+        }
+        if (st != COLI_OK) return st;
+        Launch L(m, s, "combine");
+        const int64_t n = (int64_t)T * c.hidden;
+        int grid = (int)std::min<int64_t>((n + 255) / 256, (int64_t)m->nsm * 8);
+        k_combine<<<grid, 256, 0, s>>>(m->rw, m->e_pairs, T, c.hidden, c.top_k, c.n_shared, out);
+        st = L.done();
+        if (st != COLI_OK) return st;
+    }
+    m->last_T = T;
+    return COLI_OK;
+}
+
+__global__ void k_gather_h(const int32_t *__restrict__ tok_pair, const int8_t *__restrict__ hq,
+                           const float *__restrict__ hd, int T, int slots, int I,
+                           int8_t *__restrict__ hq_out, float *__restrict__ hd_out) {
+    const int ts = blockIdx.x;  // (token, slot)
+    if (ts >= T * slots) return;
+    const int p = tok_pair[ts];
+    for (int i = threadIdx.x; i < I; i += blockDim.x) {
+        if (hq_out) hq_out[(int64_t)ts * I + i] = hq[(int64_t)p * I + i];
+        if (hd_out && i < I / COLI_QBLK) hd_out[(int64_t)ts * (I / COLI_QBLK) + i] = hd[(int64_t)p * (I / COLI_QBLK) + i];
+    }
+}
+
+}  // namespace
+
+// ===========================================================================
+extern "C" {
+
+const char *coli_status_str(coli_status s) {
+    switch (s) {
+        case COLI_OK: return "COLI_OK";
+        case COLI_EINVAL: return "COLI_EINVAL";
+        case COLI_ENOMEM: return "COLI_ENOMEM";
+        case COLI_ECUDA: return "COLI_ECUDA";
+        case COLI_EUNSUPPORTED: return "COLI_EUNSUPPORTED";
+        case COLI_ETIMEOUT: return "COLI_ETIMEOUT";
+    }
+    return "COLI_UNKNOWN";
+}
+
+const char *coli_last_error(void) { return g_last_error.c_str(); }
+int coli_abi_version(void) { return COLI_ABI_VERSION; }
+uint64_t coli_launch_count(void) { return g_launches.load(); }
+
+coli_status coli_quant_q8(const float *x, int64_t rows, int64_t len, int8_t *q, float *d,
+                          coli_stream_t stream) {
+    g_last_error.clear();
+    if (rows < 0 || len <= 0 || len % COLI_QBLK) return fail(COLI_EINVAL, "len must be a positive multiple of 32, rows >= 0");
+    if (rows == 0) return COLI_OK;
+    if (!x || !q || !d) return fail(COLI_EINVAL, "null pointer");
+    if (!aligned16(x) || !aligned16(q) || !aligned16(d)) return fail(COLI_EINVAL, "pointers must be 16-byte aligned");
+    return quant_q8_launch(nullptr, x, rows, len, q, d, (cudaStream_t)stream);
+}
+
+coli_status coli_quant_weights(const float *w, int64_t rows, int64_t K, int wfmt, void *codes,
+                               float *scales, coli_stream_t stream) {
+    g_last_error.clear();
+    if (wfmt != 8 && wfmt != 4 && wfmt != 2) return fail(COLI_EINVAL, "wfmt must be 8, 4 or 2");
+    if (rows < 0 || K <= 0 || K % (wfmt == 2 ? 64 : 32))
+        return fail(COLI_EINVAL, "K must be a positive multiple of 32 (64 for int2)");
+    if (rows == 0) return COLI_OK;
+    if (!w || !codes || !scales) return fail(COLI_EINVAL, "null pointer");
+    if (!aligned16(w) || !aligned16(codes) || !aligned16(scales)) return fail(COLI_EINVAL, "pointers must be 16-byte aligned");
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t grid = std::min<int64_t>((rows + 7) / 8, (int64_t)sm_count() * 16);
+    Launch L(nullptr, s, "quant_weights");
+    switch (wfmt) {
+        case 8: k_quant_weights<8><<<(unsigned)grid, 256, 0, s>>>(w, rows, K, (uint32_t *)codes, scales); break;
+        case 4: k_quant_weights<4><<<(unsigned)grid, 256, 0, s>>>(w, rows, K, (uint32_t *)codes, scales); break;
+        default: k_quant_weights<2><<<(unsigned)grid, 256, 0, s>>>(w, rows, K, (uint32_t *)codes, scales); break;
+    }
+    return L.done();
+}
+
+size_t coli_moe_workspace_bytes(const coli_moe_config *cfg) {
+    if (!cfg_valid(cfg, nullptr)) return 0;
+    return layout_of(*cfg).total;
+}
+
+coli_status coli_moe_create(const coli_moe_config *cfg, const float *router_w, const float *bias,
+                            const coli_expert *experts, coli_moe **out) {
+    g_last_error.clear();
+    if (!out) return fail(COLI_EINVAL, "out is NULL");
+    *out = nullptr;
+    std::string why;
+    if (!cfg_valid(cfg, &why)) return fail(COLI_EINVAL, "invalid config: %s", why.c_str());
+    if (!router_w || !bias || !experts) return fail(COLI_EINVAL, "null router/bias/experts");
+    if (!aligned16(router_w) || !aligned16(bias)) return fail(COLI_EINVAL, "router pointers must be 16-byte aligned");
+    const int n = cfg->n_routed + cfg->n_shared;
+    std::vector<ExpertDev> host(n);
+    for (int e = 0; e < n; ++e) {
+        const coli_qmat *mm[3] = {&experts[e].gate, &experts[e].up, &experts[e].down};
+        QMatDev *dd[3] = {&host[e].gate, &host[e].up, &host[e].down};
+        for (int j = 0; j < 3; ++j) {
+            if (!mm[j]->codes || !mm[j]->scales) return fail(COLI_EINVAL, "expert %d matrix %d is NULL", e, j);
+            if (!aligned16(mm[j]->codes) || !aligned16(mm[j]->scales))
+                return fail(COLI_EINVAL, "expert %d matrix %d is not 16-byte aligned", e, j);
+            dd[j]->codes = (const uint8_t *)mm[j]->codes;
+            dd[j]->scales = mm[j]->scales;
+        }
+    }
+    coli_moe *m = new (std::nothrow) coli_moe();
+    if (!m) return fail(COLI_ENOMEM, "host allocation failed");
+    m->cfg = *cfg;
+    m->router_w = router_w;
+    m->bias = bias;
+    cudaGetDevice(&m->device);
+    m->nsm = sm_count();
+    const WsOffsets o = layout_of(*cfg);
+    if (getenv("COLI_FAULT") && strcmp(getenv("COLI_FAULT"), "alloc") == 0) {
+        delete m;
+        return fail(COLI_ENOMEM, "injected allocation failure (COLI_FAULT=alloc)");
+    }
+    cudaError_t e = cudaMalloc(&m->ws_base, o.total);
+    if (e != cudaSuccess) {
+        delete m;
+        return cuda_fail(e, "cudaMalloc(workspace)");
+    }
+    m->ws_bytes = o.total;
+    char *b = (char *)m->ws_base;
+    m->rw.s = (double *)(b + o.s);
+    m->rw.c = (double *)(b + o.c);
+    m->rw.idx = (int32_t *)(b + o.idx);
+    m->rw.w = (float *)(b + o.w);
+    m->rw.bitmap = (uint32_t *)(b + o.bitmap);
+    m->rw.prefix = (int32_t *)(b + o.prefix);
+    m->rw.counter = (uint32_t *)(b + o.counter);
+    m->rw.n_active = (int32_t *)(b + o.n_active);
+    m->rw.active = (int32_t *)(b + o.active);
+    m->rw.off = (int32_t *)(b + o.off);
+    m->rw.act_of = (int32_t *)(b + o.act_of);
+    m->rw.pair_tok = (int32_t *)(b + o.pair_tok);
+    m->rw.pair_slot = (int32_t *)(b + o.pair_slot);
+    m->rw.tok_pair = (int32_t *)(b + o.tok_pair);
+    m->rw.wstride = (cfg->max_tokens + 31) / 32;
+    m->xq = (int8_t *)(b + o.xq);
+    m->xd = (float *)(b + o.xd);
+    m->hq = (int8_t *)(b + o.hq);
+    m->hd = (float *)(b + o.hd);
+    m->e_pairs = o.e_pairs ? (float *)(b + o.e_pairs) : nullptr;
+    m->x_in = (float *)(b + o.x_in);
+    m->y_out = (float *)(b + o.y_out);
+    m->experts_dev = (ExpertDev *)(b + o.experts);
+    e = cudaMemset(m->ws_base, 0, o.total);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(m->experts_dev, host.data(), sizeof(ExpertDev) * n, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        cudaFree(m->ws_base);
+        delete m;
+        return cuda_fail(e, "workspace init");
+    }
+    *out = m;
+    return COLI_OK;
+}
+
+coli_status coli_router(coli_moe *m, const float *x, int T, int32_t *idx, float *w,
+                        coli_stream_t stream) {
+    g_last_error.clear();
+    coli_status st = check_handle(m);
+    if (st != COLI_OK) return st;
+    if (T < 1 || T > m->cfg.max_tokens) return fail(COLI_EINVAL, "T=%d outside [1, max_tokens=%d]", T, m->cfg.max_tokens);
+    if (!x || !idx || !w) return fail(COLI_EINVAL, "null pointer");
+    if (!aligned16(x) || !aligned16(idx) || !aligned16(w)) return fail(COLI_EINVAL, "pointers must be 16-byte aligned");
+    return launch_route(m, x, T, idx, w, 0, (cudaStream_t)stream);
+}
+
+coli_status coli_moe_forward(coli_moe *m, const float *x, int T, float *out, coli_stream_t stream) {
+    g_last_error.clear();
+    coli_status st = check_handle(m);
+    if (st != COLI_OK) return st;
+    if (T < 1 || T > m->cfg.max_tokens) return fail(COLI_EINVAL, "T=%d outside [1, max_tokens=%d]", T, m->cfg.max_tokens);
+    if (!x || !out) return fail(COLI_EINVAL, "null pointer");
+    if (!aligned16(x) || !aligned16(out)) return fail(COLI_EINVAL, "pointers must be 16-byte aligned");
+    const size_t bytes = (size_t)T * m->cfg.hidden * 4;
+    const char *xa = (const char *)x, *oa = (const char *)out;
+    if (xa < oa + bytes && oa < xa + bytes) return fail(COLI_EINVAL, "out must not alias x");
+    return forward_impl(m, x, T, out, (cudaStream_t)stream);
+}
+
+coli_status coli_moe_forward_host(coli_moe *m, const float *x_host, int T, float *out_host,
+                                  coli_stream_t stream) {
+    g_last_error.clear();
+    coli_status st = check_handle(m);
+    if (st != COLI_OK) return st;
+    if (T < 1 || T > m->cfg.max_tokens) return fail(COLI_EINVAL, "T=%d outside [1, max_tokens=%d]", T, m->cfg.max_tokens);
+    if (!x_host || !out_host) return fail(COLI_EINVAL, "null pointer");
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t bytes = (size_t)T * m->cfg.hidden * 4;
+    COLI_CUDA(cudaMemcpyAsync(m->x_in, x_host, bytes, cudaMemcpyHostToDevice, s), "copy x in");
+    st = forward_impl(m, m->x_in, T, m->y_out, s);
+    if (st != COLI_OK) return st;
+    COLI_CUDA(cudaMemcpyAsync(out_host, m->y_out, bytes, cudaMemcpyDeviceToHost, s), "copy out");
+    COLI_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+    return COLI_OK;
+}
+
+void coli_moe_destroy(coli_moe *m) {
+    if (!m) return;
+    int prev = -1;
+    cudaGetDevice(&prev);
+    if (prev != m->device) cudaSetDevice(m->device);
+    cudaDeviceSynchronize();
+    for (auto &p : m->pending) {
+        cudaEventDestroy(p.a);
+        cudaEventDestroy(p.b);
+    }
+    for (auto e : m->event_pool) cudaEventDestroy(e);
+    cudaFree(m->ws_base);
+    if (prev >= 0 && prev != m->device) cudaSetDevice(prev);
+    delete m;
+}
+
+coli_status coli_moe_profile(coli_moe *m, int enable) {
+    g_last_error.clear();
+    if (!m) return fail(COLI_EINVAL, "handle is NULL");
+    m->profiling = enable != 0;
+    return COLI_OK;
+}
+
+coli_status coli_moe_profile_read(coli_moe *m, coli_kernel_time *out, int max_entries,
+                                  int *n_entries) {
+    g_last_error.clear();
+    if (!m || !n_entries || (max_entries > 0 && !out)) return fail(COLI_EINVAL, "bad arguments");
+    std::vector<std::pair<const char *, std::pair<int, double>>> acc;
+    for (auto &p : m->pending) {
+        float ms = 0.0f;
+        cudaError_t e = cudaEventSynchronize(p.b);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, p.a, p.b);
+        if (e != cudaSuccess) return cuda_fail(e, "profile events");
+        bool found = false;
+        for (auto &a : acc)
+            if (strcmp(a.first, p.name) == 0) {
+                a.second.first += 1;
+                a.second.second += ms;
+                found = true;
+            }
+        if (!found) acc.push_back({p.name, {1, (double)ms}});
+        m->event_pool.push_back(p.a);
+        m->event_pool.push_back(p.b);
+    }
+    m->pending.clear();
+    int n = 0;
+    for (auto &a : acc) {
+        if (n < max_entries) out[n] = coli_kernel_time{a.first, a.second.first, a.second.second};
+        ++n;
+    }
+    *n_entries = n;
+    return COLI_OK;
+}
+
+coli_status coli_dbg_block_sums(const void *codes, int wfmt, int64_t rows, int64_t K,
+                                const int8_t *xq, int T, int32_t *S, coli_stream_t stream) {
+    g_last_error.clear();
+    if (wfmt != 8 && wfmt != 4 && wfmt != 2) return fail(COLI_EINVAL, "wfmt must be 8, 4 or 2");
+    if (rows < 1 || T < 1 || T > 65535 || K <= 0 || K % (wfmt == 2 ? 64 : 32) || K > 16384)
+        return fail(COLI_EINVAL, "bad sizes");
+    if (!codes || !xq || !S) return fail(COLI_EINVAL, "null pointer");
+    if (!aligned16(codes) || !aligned16(xq) || !aligned16(S)) return fail(COLI_EINVAL, "pointers must be 16-byte aligned");
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t smem = stage_bytes(1, (int)K);
+    dim3 grid((unsigned)std::min<int64_t>((rows + 7) / 8, 1024), (unsigned)T);
+    Launch L(nullptr, s, "dbg_block_sums");
+    switch (wfmt) {
+        case 8: k_dbg_block_sums<8><<<grid, 256, smem, s>>>((const uint8_t *)codes, rows, (int)K, xq, T, S); break;
+        case 4: k_dbg_block_sums<4><<<grid, 256, smem, s>>>((const uint8_t *)codes, rows, (int)K, xq, T, S); break;
+        default: k_dbg_block_sums<2><<<grid, 256, smem, s>>>((const uint8_t *)codes, rows, (int)K, xq, T, S); break;
+    }
+    return L.done();
+}
+
+coli_status coli_dbg_last_forward(coli_moe *m, int T, int32_t *idx, float *w, int8_t *hq,
+                                  float *hd, coli_stream_t stream) {
+    g_last_error.clear();
+    coli_status st = check_handle(m);
+    if (st != COLI_OK) return st;
+    if (m->last_T == 0 || T != m->last_T) return fail(COLI_EINVAL, "T=%d does not match the last forward (T=%d)", T, m->last_T);
+    cudaStream_t s = (cudaStream_t)stream;
+    const auto &c = m->cfg;
+    if (idx) COLI_CUDA(cudaMemcpyAsync(idx, m->rw.idx, (size_t)T * c.top_k * 4, cudaMemcpyDeviceToDevice, s), "copy idx");
+    if (w) COLI_CUDA(cudaMemcpyAsync(w, m->rw.w, (size_t)T * c.top_k * 4, cudaMemcpyDeviceToDevice, s), "copy w");
+    if (hq || hd) {
+        const int slots = c.top_k + c.n_shared;
+        Launch L(nullptr, s, "dbg_gather_h");
+        k_gather_h<<<T * slots, 256, 0, s>>>(m->rw.tok_pair, m->hq, m->hd, T, slots, c.inter, hq, hd);
+        return L.done();
+    }
+    return COLI_OK;
+}
+
+}  // extern "C"

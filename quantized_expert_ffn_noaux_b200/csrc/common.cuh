@@ -1,0 +1,185 @@
+// common.cuh -- device helpers shared by the library's kernels (sm_100a).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#define COLI_QBLK 32
+
+namespace coli {
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Q8_0 of one 32-element block held one element per lane:
+// d = amax/127 (IEEE fp32 division), q = clamp(rint(x/d), -127, 127).
+__device__ __forceinline__ int q8_lane(float x, float &d_out) {
+    float amax = warp_max(fabsf(x));
+    float d = __fdiv_rn(amax, 127.0f);
+    d_out = d;
+    float v = 0.0f;
+    if (d != 0.0f) v = rintf(__fdiv_rn(x, d));
+    v = fminf(fmaxf(v, -127.0f), 127.0f);
+    return (int)v;
+}
+
+// dp4a with four unsigned 8-bit fields in a and four signed in b.
+__device__ __forceinline__ int dp4a_us(unsigned a, int b, int c) {
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ int dp4a_ss(int a, int b, int c) {
+    int d;
+    asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// ---------------------------------------------------------------------------
+// Activation staging.  A weight row of K elements is read as V = K*BITS/128
+// uint4 vectors.  For vector v the activation codes it multiplies are stored
+// in shared memory as P = 4/ (BITS/2) ... planes of 16 bytes, arranged so the
+// unpacked weight fields line up with dp4a operands:
+//   BITS 8: plane 0 holds x[16v .. 16v+15] in natural order          (P = 1)
+//   BITS 4: vector v is block v; weight word i (elements 8i..8i+7 of the
+//           block) unpacks into low nibbles (elements 8i+0,2,4,6) and high
+//           nibbles (8i+1,3,5,7); the activation words are stored
+//           [E0 O0 E1 O1] in plane 0 and [E2 O2 E3 O3] in plane 1        (P = 2)
+//   BITS 2: vector v covers blocks 2v, 2v+1; weight word i holds elements
+//           16i + 4j + f in byte j, bits 2f..2f+1; plane i stores the four
+//           words G_f = (x[16i+f], x[16i+4+f], x[16i+8+f], x[16i+12+f])  (P = 4)
+// Plane p of a row of V vectors starts at p*V*16 bytes.
+template <int BITS> struct Fmt {
+    static constexpr int ELEMS = 128 / BITS;       // elements per uint4 of weights
+    static constexpr int PLANES = ELEMS / 16;      // 16-byte activation planes per uint4
+    static constexpr int OFFSET = BITS == 8 ? 0 : (BITS == 4 ? 8 : 2);  // unsigned bias
+};
+
+// Byte (element index within the vector's ELEMS) that activation byte
+// `pos` (0 .. ELEMS-1, plane-major) must hold.
+template <int BITS> __device__ __forceinline__ int stage_src(int pos) {
+    if (BITS == 8) return pos;
+    if (BITS == 4) {
+        int plane = pos >> 4, w = (pos >> 2) & 3, byte = pos & 3;
+        int word = plane * 2 + (w >> 1);  // weight word 0..3
+        int odd = w & 1;
+        return word * 8 + byte * 2 + odd;
+    }
+    // BITS == 2
+    int word = pos >> 4, f = (pos >> 2) & 3, byte = pos & 3;
+    return word * 16 + byte * 4 + f;
+}
+
+// Integer partial dot of one weight vector with its staged activations.
+// Returns the raw dp4a sums for each 32-block fragment the vector covers
+// (one for BITS 8 -- half a block -- and 4, two for BITS 2), before the
+// unsigned-offset correction.
+template <int BITS>
+__device__ __forceinline__ void vec_dot(const uint4 w, const uint4 *act, int V, int &s0, int &s1) {
+    if (BITS == 8) {
+        uint4 a = act[0];
+        int s = 0;
+        s = dp4a_ss((int)w.x, (int)a.x, s);
+        s = dp4a_ss((int)w.y, (int)a.y, s);
+        s = dp4a_ss((int)w.z, (int)a.z, s);
+        s = dp4a_ss((int)w.w, (int)a.w, s);
+        s0 = s;
+        s1 = 0;
+    } else if (BITS == 4) {
+        uint4 a0 = act[0], a1 = act[V];
+        unsigned t0 = w.x ^ 0x88888888u, t1 = w.y ^ 0x88888888u;
+        unsigned t2 = w.z ^ 0x88888888u, t3 = w.w ^ 0x88888888u;
+        int s = 0;
+        s = dp4a_us(t0 & 0x0F0F0F0Fu, (int)a0.x, s);
+        s = dp4a_us((t0 >> 4) & 0x0F0F0F0Fu, (int)a0.y, s);
+        s = dp4a_us(t1 & 0x0F0F0F0Fu, (int)a0.z, s);
+        s = dp4a_us((t1 >> 4) & 0x0F0F0F0Fu, (int)a0.w, s);
+        s = dp4a_us(t2 & 0x0F0F0F0Fu, (int)a1.x, s);
+        s = dp4a_us((t2 >> 4) & 0x0F0F0F0Fu, (int)a1.y, s);
+        s = dp4a_us(t3 & 0x0F0F0F0Fu, (int)a1.z, s);
+        s = dp4a_us((t3 >> 4) & 0x0F0F0F0Fu, (int)a1.w, s);
+        s0 = s;
+        s1 = 0;
+    } else {
+        uint4 a0 = act[0], a1 = act[V], a2 = act[2 * V], a3 = act[3 * V];
+        unsigned t0 = w.x ^ 0xAAAAAAAAu, t1 = w.y ^ 0xAAAAAAAAu;
+        unsigned t2 = w.z ^ 0xAAAAAAAAu, t3 = w.w ^ 0xAAAAAAAAu;
+        int s = 0, u = 0;
+        s = dp4a_us(t0 & 0x03030303u, (int)a0.x, s);
+        s = dp4a_us((t0 >> 2) & 0x03030303u, (int)a0.y, s);
+        s = dp4a_us((t0 >> 4) & 0x03030303u, (int)a0.z, s);
+        s = dp4a_us((t0 >> 6) & 0x03030303u, (int)a0.w, s);
+        s = dp4a_us(t1 & 0x03030303u, (int)a1.x, s);
+        s = dp4a_us((t1 >> 2) & 0x03030303u, (int)a1.y, s);
+        s = dp4a_us((t1 >> 4) & 0x03030303u, (int)a1.z, s);
+        s = dp4a_us((t1 >> 6) & 0x03030303u, (int)a1.w, s);
+        u = dp4a_us(t2 & 0x03030303u, (int)a2.x, u);
+        u = dp4a_us((t2 >> 2) & 0x03030303u, (int)a2.y, u);
+        u = dp4a_us((t2 >> 4) & 0x03030303u, (int)a2.z, u);
+        u = dp4a_us((t2 >> 6) & 0x03030303u, (int)a2.w, u);
+        u = dp4a_us(t3 & 0x03030303u, (int)a3.x, u);
+        u = dp4a_us((t3 >> 2) & 0x03030303u, (int)a3.y, u);
+        u = dp4a_us((t3 >> 4) & 0x03030303u, (int)a3.z, u);
+        u = dp4a_us((t3 >> 6) & 0x03030303u, (int)a3.w, u);
+        s0 = s;
+        s1 = u;
+    }
+}
+
+// fp64 promotion of vector v's partial sums: acc += sum_frag S_frag * d_block.
+// xs[b] is the sum of the activation codes of block b (for the offset
+// correction), xd[b] its Q8_0 scale.
+template <int BITS>
+__device__ __forceinline__ double vec_promote(int v, int s0, int s1, const int *xs,
+                                              const float *xd, double acc) {
+    if (BITS == 8) {
+        acc = fma((double)s0, (double)xd[v >> 1], acc);
+    } else if (BITS == 4) {
+        int S = s0 - 8 * xs[v];
+        acc = fma((double)S, (double)xd[v], acc);
+    } else {
+        int S0 = s0 - 2 * xs[2 * v], S1 = s1 - 2 * xs[2 * v + 1];
+        acc = fma((double)S0, (double)xd[2 * v], acc);
+        acc = fma((double)S1, (double)xd[2 * v + 1], acc);
+    }
+    return acc;
+}
+
+// Block sums of the vector's fragments after the offset correction
+// (exact int32; used by the parity export).
+template <int BITS>
+__device__ __forceinline__ void vec_block_sums(int v, int s0, int s1, const int *xs, int &b0,
+                                               int &S0, int &b1, int &S1) {
+    if (BITS == 8) {
+        b0 = v >> 1; S0 = s0; b1 = -1; S1 = 0;
+    } else if (BITS == 4) {
+        b0 = v; S0 = s0 - 8 * xs[v]; b1 = -1; S1 = 0;
+    } else {
+        b0 = 2 * v; S0 = s0 - 2 * xs[2 * v];
+        b1 = 2 * v + 1; S1 = s1 - 2 * xs[2 * v + 1];
+    }
+}
+
+}  // namespace coli
