@@ -49,6 +49,8 @@ def parse():
     p.add_argument("--tokens", type=int, default=None, help="override tokens per step")
     p.add_argument("--bits", type=int, default=None, choices=[8, 4, 2])
     p.add_argument("--layers", type=int, default=8)
+    p.add_argument("--n-routed", type=int, default=None,
+                   help="override the routed expert count (smaller layers for profiling)")
     p.add_argument("--e2e-steps", type=int, default=2000)
     p.add_argument("--profile-steps", type=int, default=400)
     p.add_argument("--cpu-sample-tokens", type=int, default=8)
@@ -435,6 +437,8 @@ def main():
         over["tokens"] = args.tokens
     if args.bits is not None:
         over["bits"] = args.bits
+    if args.n_routed is not None:
+        over["n_routed"] = args.n_routed
     cfg = synth.workload(args.workload, **over)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

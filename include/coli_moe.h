@@ -159,6 +159,13 @@ void coli_moe_destroy(coli_moe *m);
 /* Bytes of device workspace coli_moe_create would allocate (0 if cfg is invalid). */
 size_t coli_moe_workspace_bytes(const coli_moe_config *cfg);
 
+/* Synchronise `stream` and report device-side failures of earlier calls on
+ * this handle: every wait inside the library's kernels is bounded (about one
+ * second); a wait that gives up records COLI_ETIMEOUT in the handle's error
+ * word and its kernel returns early, leaving that call's outputs undefined.
+ * Returns COLI_ETIMEOUT (and clears the word) if that happened, else COLI_OK. */
+coli_status coli_moe_device_status(coli_moe *m, coli_stream_t stream);
+
 /* Kernel launches made by this library in this process so far. */
 uint64_t coli_launch_count(void);
 
@@ -192,6 +199,13 @@ coli_status coli_dbg_block_sums(const void *codes, int wfmt, int64_t rows, int64
  *   fp32 (device).  Any output may be NULL.  T must equal that call's T. */
 coli_status coli_dbg_last_forward(coli_moe *m, int T, int32_t *idx, float *w, int8_t *hq,
                                   float *hd, coli_stream_t stream);
+
+/* Test hook for the bounded waits (no counterpart on the pages): one thread
+ * waits on an mbarrier that nothing ever arrives at, through the same bounded
+ * wait the pipelined kernels use.  The wait gives up after about one second
+ * and records COLI_ETIMEOUT in the handle's error word, which the next
+ * coli_moe_device_status reports.  Nothing faults or hangs. */
+coli_status coli_dbg_wait_probe(coli_moe *m, coli_stream_t stream);
 
 #ifdef __cplusplus
 }

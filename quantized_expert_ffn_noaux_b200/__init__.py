@@ -79,6 +79,8 @@ def lib():
         "coli_moe_profile_read": ([vp, vp, ci, ctypes.POINTER(ci)], ci),
         "coli_dbg_block_sums": ([vp, ci, i64, i64, vp, ci, vp, vp], ci),
         "coli_dbg_last_forward": ([vp, ci, vp, vp, vp, vp, vp], ci),
+        "coli_dbg_wait_probe": ([vp, vp], ci),
+        "coli_moe_device_status": ([vp, vp], ci),
     }
     for name, (args, res) in sigs.items():
         f = getattr(L, name)
@@ -230,6 +232,13 @@ class MoELayer:
         n = ctypes.c_int()
         _check(lib().coli_moe_profile_read(self._h, arr, 32, ctypes.byref(n)))
         return {arr[i].name.decode(): (arr[i].launches, arr[i].ms) for i in range(min(n.value, 32))}
+
+    def device_status(self, stream=None):
+        """Synchronise and return the device-side status (COLI_OK or COLI_ETIMEOUT)."""
+        return int(lib().coli_moe_device_status(self._h, _stream(stream)))
+
+    def dbg_wait_probe(self, stream=None):
+        _check(lib().coli_dbg_wait_probe(self._h, _stream(stream)))
 
     def dbg_last_forward(self, T, stream=None):
         c = self.cfg

@@ -95,6 +95,8 @@ struct coli_moe {
     float *hd = nullptr;
     float *e_pairs = nullptr;  // only when max_tokens > SMALL_T
     float *x_in = nullptr, *y_out = nullptr;
+    uint8_t *xrec = nullptr, *hrec = nullptr;
+    int *err = nullptr;
     int last_T = 0;
     std::map<const void *, int> occ_cache;  // kernel -> CTAs per SM (attributes already set)
     // profiling
@@ -116,7 +118,7 @@ struct Layout {
 
 struct WsOffsets {
     size_t s, c, idx, w, bitmap, prefix, counter, n_active, active, off, act_of, pair_tok,
-        pair_slot, tok_pair, xq, xd, hq, hd, e_pairs, x_in, y_out, experts;
+        pair_slot, tok_pair, xq, xd, hq, hd, e_pairs, x_in, y_out, experts, xrec, hrec, err;
     size_t total;
 };
 
@@ -173,6 +175,9 @@ WsOffsets layout_of(const coli_moe_config &c) {
     o.x_in = L.add(T * H * 4);
     o.y_out = L.add(T * H * 4);
     o.experts = L.add((E + S) * sizeof(ExpertDev));
+    o.xrec = L.add(T * (size_t)rec_bytes((int)H));
+    o.hrec = L.add(P * (size_t)rec_bytes((int)I));
+    o.err = L.add(4);
     o.total = L.total;
     return o;
 }
@@ -342,14 +347,161 @@ coli_status launch_down_grouped(coli_moe *m, int max_items, cudaStream_t s) {
     }
 }
 
-size_t select_smem(const coli_moe_config &c) {
-    return (size_t)c.n_routed * 8 + (size_t)c.n_group * 12 + (size_t)c.top_k * 4 + 16;
+size_t select_smem(const coli_moe_config &c) { return select_smem_bytes(c.n_routed, c.n_group); }
+
+// Launch with programmatic stream serialization (PDL) when `pdl` is set: the
+// kernel may start while the previous kernel on the stream is finishing and
+// waits for it with griddepcontrol.wait before reading its results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t s, bool pdl, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// ---- few-token path sizing ------------------------------------------------
+constexpr int SMEM_BUDGET = 227 * 1024;
+
+struct PipePlan {
+    int ns = 0;            // ring stages
+    size_t stage = 0;      // bytes per stage
+    size_t smem = 0;       // dynamic shared memory
+    int stage_rows = 0;    // down: rows per stage
+    int grid = 0;
+    int rows_cap = 0;      // down: rows per CTA (max)
+    int amax = 0, pmax = 0;
+};
+
+int ring_stages(size_t fixed, size_t stage) {
+    if (fixed >= (size_t)SMEM_BUDGET) return 0;
+    return (int)std::min<size_t>((SMEM_BUDGET - fixed) / stage, PIPE_MAX_STAGES);
+}
+
+PipePlan plan_gateup(const coli_moe *m, int T) {
+    const auto &c = m->cfg;
+    PipePlan p;
+    const int RB = c.hidden * c.wfmt / 8;
+    const int R = pipe_rows_per_stage(RB);
+    const int slices = R >= PIPE_CONSUMERS ? 1 : PIPE_CONSUMERS / R;
+    p.amax = std::min(c.n_routed, T * c.top_k) + c.n_shared;
+    p.pmax = T * (c.top_k + c.n_shared);
+    p.stage = (size_t)R * RB;
+    const size_t fixed = pipe_hdr_bytes() + align128((size_t)(2 * p.amax + 1 + p.pmax) * 4) +
+                         align128((size_t)T * rec_bytes(c.hidden)) +
+                         (size_t)2 * 2 * 32 * slices * PIPE_MAX_TOK * 8;
+    p.ns = ring_stages(fixed, p.stage);
+    p.smem = fixed + (size_t)p.ns * p.stage;
+    p.grid = std::max(1, std::min(m->nsm, p.amax * (c.inter / 32)));
+    return p;
+}
+
+PipePlan plan_down(const coli_moe *m, int T) {
+    const auto &c = m->cfg;
+    PipePlan p;
+    const int RB = c.inter * c.wfmt / 8;
+    p.grid = std::min(m->nsm, c.hidden);
+    p.rows_cap = (c.hidden + p.grid - 1) / p.grid;
+    p.stage_rows = std::max(1, std::min(p.rows_cap, PIPE_STAGE_MAX / RB));
+    p.stage = (size_t)p.stage_rows * RB;
+    p.pmax = T * (c.top_k + c.n_shared);
+    const size_t fixed = pipe_hdr_bytes() + align128((size_t)p.pmax * rec_bytes(c.inter)) +
+                         (size_t)p.pmax * p.rows_cap * 4;
+    p.ns = ring_stages(fixed, p.stage);
+    p.smem = fixed + (size_t)p.ns * p.stage;
+    return p;
+}
+
+bool small_path_ok(const coli_moe *m, int T) {
+    if (T > PIPE_MAX_TOK) return false;
+    return plan_gateup(m, T).ns >= 2 && plan_down(m, T).ns >= 2;
+}
+
+template <int BITS>
+coli_status launch_small_path(coli_moe *m, const float *x, int T, float *out, cudaStream_t s) {
+    const auto &c = m->cfg;
+    coli_status st;
+    {   // router + Q8_0(x) records + selection + union
+        const size_t smem = select_smem(c) + 4 * (size_t)c.n_routed + 4 * (size_t)T * c.top_k;
+        int occ = 1;
+        void (*kern)(const float *, int, int, const float *, const float *, int, int, int, int,
+                     int, float, RouteWs, uint8_t *, int8_t *, float *, int, int32_t *, float *);
+        if (T <= 1) kern = k_router_small<1, BITS>;
+        else if (T <= 2) kern = k_router_small<2, BITS>;
+        else if (T <= 4) kern = k_router_small<4, BITS>;
+        else kern = k_router_small<8, BITS>;
+        st = prepare(m, kern, 256, smem, &occ);
+        if (st != COLI_OK) return st;
+        Launch L(m, s, "router");
+        kern<<<c.n_routed, 256, smem, s>>>(x, T, c.hidden, m->router_w, m->bias, c.n_routed,
+                                           c.n_shared, c.n_group, c.topk_group, c.top_k,
+                                           c.routed_scaling_factor, m->rw, m->xrec, m->xq, m->xd,
+                                           1, m->rw.idx, m->rw.w);
+        st = L.done();
+        if (st != COLI_OK) return st;
+    }
+    {   // gate/up + SwiGLU + Q8_0(h)
+        const PipePlan p = plan_gateup(m, T);
+        auto kern = k_gateup_pipe<BITS>;
+        int occ = 1;
+        st = prepare(m, kern, PIPE_THREADS, p.smem, &occ);
+        if (st != COLI_OK) return st;
+        Launch L(m, s, "gateup_pipe");
+        cudaError_t e = launch_ex(kern, dim3(p.grid), dim3(PIPE_THREADS), p.smem, s, true, m->rw,
+                                  (const ExpertDev *)m->experts_dev, (const uint8_t *)m->xrec, T,
+                                  c.hidden, c.inter, p.ns, p.amax, p.pmax, m->hrec, m->hq, m->hd,
+                                  m->err);
+        if (e != cudaSuccess) return cuda_fail(e, "gateup_pipe launch");
+        st = L.done();
+        if (st != COLI_OK) return st;
+    }
+    {   // down + combine
+        const PipePlan p = plan_down(m, T);
+        auto kern = k_down_pipe<BITS>;
+        int occ = 1;
+        st = prepare(m, kern, PIPE_THREADS, p.smem, &occ);
+        if (st != COLI_OK) return st;
+        Launch L(m, s, "down_pipe");
+        cudaError_t e = launch_ex(kern, dim3(p.grid), dim3(PIPE_THREADS), p.smem, s, true, m->rw,
+                                  (const ExpertDev *)m->experts_dev, (const uint8_t *)m->hrec, T,
+                                  c.hidden, c.inter, c.top_k, c.n_shared, p.ns, p.stage_rows,
+                                  p.rows_cap, out, m->err);
+        if (e != cudaSuccess) return cuda_fail(e, "down_pipe launch");
+        st = L.done();
+        if (st != COLI_OK) return st;
+    }
+    return COLI_OK;
 }
 
 coli_status launch_route(coli_moe *m, const float *x, int T, int32_t *idx, float *w,
                          int do_union, cudaStream_t s) {
     const auto &c = m->cfg;
     const int E = c.n_routed, H = c.hidden;
+    if (T <= 8 && !do_union) {
+        const size_t smem = select_smem(c) + 4 * (size_t)c.n_routed + 4 * (size_t)T * c.top_k;
+        int occ = 1;
+        void (*kern)(const float *, int, int, const float *, const float *, int, int, int, int,
+                     int, float, RouteWs, uint8_t *, int8_t *, float *, int, int32_t *, float *);
+        if (T <= 1) kern = k_router_small<1, 4>;
+        else if (T <= 2) kern = k_router_small<2, 4>;
+        else if (T <= 4) kern = k_router_small<4, 4>;
+        else kern = k_router_small<8, 4>;
+        coli_status st = prepare(m, kern, 256, smem, &occ);
+        if (st != COLI_OK) return st;
+        Launch L(m, s, "router");
+        kern<<<E, 256, smem, s>>>(x, T, H, m->router_w, m->bias, E, c.n_shared, c.n_group,
+                                  c.topk_group, c.top_k, c.routed_scaling_factor, m->rw, nullptr,
+                                  nullptr, nullptr, 0, idx, w);
+        return L.done();
+    }
     {
         Launch L(m, s, "router_logits");
         if (T <= 8) {
@@ -404,6 +556,15 @@ coli_status check_handle(coli_moe *m) {
 coli_status forward_impl(coli_moe *m, const float *x, int T, float *out, cudaStream_t s) {
     const auto &c = m->cfg;
     coli_status st;
+    if (small_path_ok(m, T)) {
+        switch (c.wfmt) {
+            case 8: st = launch_small_path<8>(m, x, T, out, s); break;
+            case 4: st = launch_small_path<4>(m, x, T, out, s); break;
+            default: st = launch_small_path<2>(m, x, T, out, s); break;
+        }
+        if (st == COLI_OK) m->last_T = T;
+        return st;
+    }
     st = quant_q8_launch(m, x, T, c.hidden, m->xq, m->xd, s);
     if (st != COLI_OK) return st;
     st = launch_route(m, x, T, m->rw.idx, m->rw.w, 1, s);
@@ -443,6 +604,16 @@ coli_status forward_impl(coli_moe *m, const float *x, int T, float *out, cudaStr
     }
     m->last_T = T;
     return COLI_OK;
+}
+
+__global__ void k_dbg_wait_probe(int *err) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, err);  // nothing arrives: gives up
 }
 
 __global__ void k_gather_h(const int32_t *__restrict__ tok_pair, const int8_t *__restrict__ hq,
@@ -577,6 +748,9 @@ coli_status coli_moe_create(const coli_moe_config *cfg, const float *router_w, c
     m->x_in = (float *)(b + o.x_in);
     m->y_out = (float *)(b + o.y_out);
     m->experts_dev = (ExpertDev *)(b + o.experts);
+    m->xrec = (uint8_t *)(b + o.xrec);
+    m->hrec = (uint8_t *)(b + o.hrec);
+    m->err = (int *)(b + o.err);
     e = cudaMemset(m->ws_base, 0, o.total);
     if (e == cudaSuccess)
         e = cudaMemcpy(m->experts_dev, host.data(), sizeof(ExpertDev) * n, cudaMemcpyHostToDevice);
@@ -682,6 +856,32 @@ coli_status coli_moe_profile_read(coli_moe *m, coli_kernel_time *out, int max_en
     }
     *n_entries = n;
     return COLI_OK;
+}
+
+coli_status coli_moe_device_status(coli_moe *m, coli_stream_t stream) {
+    g_last_error.clear();
+    coli_status st = check_handle(m);
+    if (st != COLI_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    int word = 0;
+    COLI_CUDA(cudaMemcpyAsync(&word, m->err, sizeof(int), cudaMemcpyDeviceToHost, s), "read error word");
+    COLI_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+    if (word != 0) {
+        COLI_CUDA(cudaMemsetAsync(m->err, 0, sizeof(int), s), "clear error word");
+        COLI_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+        return fail(COLI_ETIMEOUT, "a device-side wait gave up (error word %d)", word);
+    }
+    return COLI_OK;
+}
+
+coli_status coli_dbg_wait_probe(coli_moe *m, coli_stream_t stream) {
+    g_last_error.clear();
+    coli_status st = check_handle(m);
+    if (st != COLI_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    Launch L(nullptr, s, "dbg_wait_probe");
+    k_dbg_wait_probe<<<1, 32, 0, s>>>(m->err);
+    return L.done();
 }
 
 coli_status coli_dbg_block_sums(const void *codes, int wfmt, int64_t rows, int64_t K,

@@ -183,3 +183,142 @@ __device__ __forceinline__ void vec_block_sums(int v, int s0, int s1, const int 
 }
 
 }  // namespace coli
+
+// ---------------------------------------------------------------------------
+// Asynchronous bulk copies (cp.async.bulk, the non-tensor TMA path) into
+// shared memory, completed on mbarriers; every wait is bounded.
+namespace coli {
+
+// A wait that has not completed after this many SM cycles (~1 s) gives up:
+// the kernel records COLI_ETIMEOUT (5) in its error word and returns.
+constexpr long long WAIT_LIMIT_CYCLES = 2000000000LL;
+constexpr int ERR_TIMEOUT = 5;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity; false (and the error
+// word set) if it did not complete within WAIT_LIMIT_CYCLES.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+            if (err) atomicExch(err, ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// Global -> shared bulk copy of `bytes` (multiple of 16, both addresses
+// 16-byte aligned), completing transaction bytes on `bar`.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
+                                         uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Programmatic dependent launch: wait for the preceding grid's completion and
+// memory flush; allow the next grid to start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Named barrier among `nthreads` threads (a multiple of 32), id 1..15.
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Activation records.  One Q8_0 row of length K prepared for a weight format:
+//   [0, K)            codes in the staged plane layout of Fmt<BITS>
+//   [K, K + 4nb)      int32 sums of the codes of each 32-block
+//   [K + 4nb, K + 8nb) fp32 Q8_0 scales
+// padded to a multiple of 16 bytes.
+__host__ __device__ inline int rec_bytes(int K) {
+    return ((K + 8 * (K / COLI_QBLK)) + 15) & ~15;
+}
+
+// Byte offset inside the record's code area and the element (0..31 within
+// block b) that lane position i of block b holds, for a row of V vectors.
+template <int BITS>
+__device__ __forceinline__ void rec_slot(int b, int i, int V, int &offset, int &src) {
+    if (BITS == 8) {
+        const int v = 2 * b + (i >> 4);
+        offset = v * 16 + (i & 15);
+        src = i;
+    } else if (BITS == 4) {
+        const int v = b, P = i;
+        offset = (P >> 4) * V * 16 + v * 16 + (P & 15);
+        src = stage_src<4>(P);
+    } else {
+        const int v = b >> 1, h = b & 1, P = 32 * h + i;
+        offset = (P >> 4) * V * 16 + v * 16 + (P & 15);
+        src = stage_src<2>(P) - 32 * h;
+    }
+}
+
+// Q8_0 of one 32-block held one element per lane, written into a record:
+// codes at their staged positions, the block's code sum and scale.
+// Optionally also the natural-order codes and scale (q_nat, d_nat).
+template <int BITS>
+__device__ __forceinline__ void q8_block_to_record(float x, int b, int K, uint8_t *rec,
+                                                   int8_t *q_nat, float *d_nat) {
+    const int lane = threadIdx.x & 31;
+    float d;
+    const int code = q8_lane(x, d);
+    const int sum = warp_sum_i(code);
+    const int V = K * BITS / 128;
+    int off, src;
+    rec_slot<BITS>(b, lane, V, off, src);
+    const int mine = __shfl_sync(0xffffffffu, code, src);
+    rec[off] = (uint8_t)(int8_t)mine;
+    if (lane == 0) {
+        const int nb = K / COLI_QBLK;
+        reinterpret_cast<int *>(rec + K)[b] = sum;
+        reinterpret_cast<float *>(rec + K + 4 * nb)[b] = d;
+    }
+    if (q_nat) q_nat[b * COLI_QBLK + lane] = (int8_t)code;
+    if (d_nat && lane == 0) d_nat[b] = d;
+}
+
+}  // namespace coli

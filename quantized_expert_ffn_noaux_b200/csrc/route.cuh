@@ -148,71 +148,127 @@ __device__ __forceinline__ int block_exscan256(int v, int *tmp /*[8]*/, int &tot
     return base + inc - v;
 }
 
-// One CTA (256 threads) per token: group scores, group and expert ranks,
-// renormalised weights.  With `do_union`, the experts are also marked in the
-// membership bitmap and the last CTA to finish builds the batch-union tables.
-__global__ void __launch_bounds__(256) k_route_select(
-    RouteWs ws, int T, int E, int S, int G, int gk, int k, float rsf, int32_t *__restrict__ idx_out,
-    float *__restrict__ w_out, int do_union) {
-    extern __shared__ double smem_d[];
-    double *c_s = smem_d;                 // [E]
-    double *gscore = c_s + E;             // [G]
-    int *keep = (int *)(gscore + G);      // [G]
-    int *sel = keep + G;                  // [k]
-    __shared__ int is_last;
-    __shared__ int scan_tmp[8];
-    const int t = blockIdx.x, tid = threadIdx.x;
+// ---------------------------------------------------------------------------
+// Selection of one token by a whole CTA (256 threads), rank based, no serial
+// scans:  in-group ranks give each group's two best c (its score); group
+// ranks keep the topk_group best groups; the top_k of the kept experts are
+// among the experts ranked < top_k inside their own kept group, and their
+// ranks among those candidates give idx sorted by descending c.  Every
+// comparison breaks ties toward the lower index.
+struct SelectSmem {
+    double *c;      // [E]
+    double *s;      // [E]
+    int *grank;     // [E] rank inside its group
+    double *top1;   // [G]
+    double *top2;   // [G]
+    int *keep;      // [G]
+    int *cand;      // [E]
+    int *ncand;     // [1]
+    int *sel;       // [32]
+};
+
+__host__ __device__ inline size_t select_smem_bytes(int E, int G) {
+    return (size_t)E * 16 + (size_t)G * 16 + (size_t)E * 8 + (size_t)G * 4 + 4 + 32 * 4 + 64;
+}
+
+__device__ inline SelectSmem carve_select(void *base, int E, int G) {
+    SelectSmem m;
+    char *p = (char *)base;
+    m.c = (double *)p;           p += (size_t)E * 8;
+    m.s = (double *)p;           p += (size_t)E * 8;
+    m.top1 = (double *)p;        p += (size_t)G * 8;
+    m.top2 = (double *)p;        p += (size_t)G * 8;
+    m.grank = (int *)p;          p += (size_t)E * 4;
+    m.cand = (int *)p;           p += (size_t)E * 4;
+    m.keep = (int *)p;           p += (size_t)G * 4;
+    m.ncand = (int *)p;          p += 4;
+    m.sel = (int *)p;
+    return m;
+}
+
+__device__ void cta_select_token(const double *c_row, const double *s_row, int E, int G, int gk,
+                                 int k, float rsf, const SelectSmem &sm, int32_t *idx_out,
+                                 float *w_out) {
+    const int tid = threadIdx.x, nthr = blockDim.x;
     const int per = E / G;
-    const double *c_t = ws.c + (int64_t)t * E;
-    for (int e = tid; e < E; e += 256) c_s[e] = c_t[e];
+    for (int e = tid; e < E; e += nthr) {
+        sm.c[e] = __ldcg(c_row + e);
+        sm.s[e] = __ldcg(s_row + e);
+    }
+    if (tid == 0) *sm.ncand = 0;
     __syncthreads();
-    for (int g = tid; g < G; g += 256) {
-        int b1 = -1, b2 = -1;
+    for (int e = tid; e < E; e += nthr) {
+        const int g = e / per;
+        const double v = sm.c[e];
+        int r = 0;
         for (int i = 0; i < per; ++i) {
-            int e = g * per + i;
-            if (b1 < 0 || c_s[e] > c_s[b1]) b1 = e;
+            const int f = g * per + i;
+            const double u = sm.c[f];
+            r += (u > v) || (u == v && f < e);
         }
-        for (int i = 0; i < per; ++i) {
-            int e = g * per + i;
-            if (e == b1) continue;
-            if (b2 < 0 || c_s[e] > c_s[b2]) b2 = e;
-        }
-        gscore[g] = c_s[b1] + (b2 >= 0 ? c_s[b2] : 0.0);
+        sm.grank[e] = r;
+        if (r == 0) sm.top1[g] = v;
+        if (r == 1) sm.top2[g] = v;
     }
     __syncthreads();
-    for (int g = tid; g < G; g += 256) {
-        int rank = 0;
-        double v = gscore[g];
+    for (int g = tid; g < G; g += nthr) {
+        const double v = sm.top1[g] + (per > 1 ? sm.top2[g] : 0.0);
+        sm.top2[g] = v;  // reuse: group score
+    }
+    __syncthreads();
+    for (int g = tid; g < G; g += nthr) {
+        const double v = sm.top2[g];
+        int r = 0;
         for (int h = 0; h < G; ++h) {
-            double u = gscore[h];
-            rank += (u > v) || (u == v && h < g);
+            const double u = sm.top2[h];
+            r += (u > v) || (u == v && h < g);
         }
-        keep[g] = rank < gk;
+        sm.keep[g] = r < gk;
     }
     __syncthreads();
-    for (int e = tid; e < E; e += 256) {
-        if (!keep[e / per]) continue;
-        int rank = 0;
-        double v = c_s[e];
-        for (int f = 0; f < E; ++f) {
-            if (!keep[f / per]) continue;
-            double u = c_s[f];
-            rank += (u > v) || (u == v && f < e);
+    for (int e = tid; e < E; e += nthr)
+        if (sm.keep[e / per] && sm.grank[e] < k) sm.cand[atomicAdd(sm.ncand, 1)] = e;
+    __syncthreads();
+    const int n = *sm.ncand;
+    for (int i = tid; i < n; i += nthr) {
+        const int e = sm.cand[i];
+        const double v = sm.c[e];
+        int r = 0;
+        for (int j = 0; j < n; ++j) {
+            const int f = sm.cand[j];
+            const double u = sm.c[f];
+            r += (u > v) || (u == v && f < e);
         }
-        if (rank < k) sel[rank] = e;
+        if (r < k) sm.sel[r] = e;
     }
     __syncthreads();
     if (tid == 0) {
-        const double *s_t = ws.s + (int64_t)t * E;
         double ssum = 0.0;
-        for (int j = 0; j < k; ++j) ssum += s_t[sel[j]];
+        for (int j = 0; j < k; ++j) ssum += sm.s[sm.sel[j]];
         for (int j = 0; j < k; ++j) {
-            int e = sel[j];
-            float wj = (float)((s_t[e] / ssum) * (double)rsf);
-            idx_out[(int64_t)t * k + j] = e;
-            w_out[(int64_t)t * k + j] = wj;
+            const int e = sm.sel[j];
+            idx_out[j] = e;
+            w_out[j] = (float)((sm.s[e] / ssum) * (double)rsf);
         }
     }
+    __syncthreads();
+}
+
+// One CTA (256 threads) per token: cta_select_token.  With `do_union`, the
+// experts are also marked in the membership bitmap and the last CTA to finish
+// builds the batch-union tables.  Dynamic smem: select_smem_bytes(E, G).
+__global__ void __launch_bounds__(256) k_route_select(
+    RouteWs ws, int T, int E, int S, int G, int gk, int k, float rsf, int32_t *__restrict__ idx_out,
+    float *__restrict__ w_out, int do_union) {
+    extern __shared__ __align__(16) double smem_d[];
+    __shared__ int is_last;
+    __shared__ int scan_tmp[8];
+    const int t = blockIdx.x, tid = threadIdx.x;
+    const SelectSmem sm = carve_select(smem_d, E, G);
+    cta_select_token(ws.c + (int64_t)t * E, ws.s + (int64_t)t * E, E, G, gk, k, rsf, sm,
+                     idx_out + (int64_t)t * k, w_out + (int64_t)t * k);
+    double *c_s = sm.c;
+    const int *sel = idx_out + (int64_t)t * k;
     if (!do_union) return;
     if (tid < k) atomicOr(ws.bitmap + (int64_t)sel[tid] * ws.wstride + (t >> 5), 1u << (t & 31));
     __threadfence();
@@ -286,6 +342,169 @@ __global__ void __launch_bounds__(256) k_route_select(
     __syncthreads();
     for (int i = tid; i < E * nw; i += 256) ws.bitmap[(int64_t)(i / nw) * ws.wstride + (i % nw)] = 0u;
     if (tid == 0) *ws.counter = 0u;
+}
+
+
+// Batch-union tables for few tokens (T * k <= 256), built by one CTA from
+// idx [T][k]: active experts ascending (shared experts last), each expert's
+// tokens in token order.
+__device__ void cta_union_small(RouteWs ws, const int32_t *idx_g, int T, int E, int S, int k,
+                                int *cnt /*smem [E]*/, int *idx /*smem [T*k]*/,
+                                int *scan_tmp /*smem [8]*/) {
+    const int tid = threadIdx.x;
+    for (int i = tid; i < T * k; i += 256) idx[i] = idx_g[i];
+    __syncthreads();
+    for (int e = tid; e < E; e += 256) {
+        int c = 0;
+        for (int i = 0; i < T * k; ++i) c += (idx[i] == e);
+        cnt[e] = c;
+    }
+    __syncthreads();
+    int na_base = 0, pair_base = 0;
+    for (int e0 = 0; e0 < E; e0 += 256) {
+        const int e = e0 + tid;
+        const int c = (e < E) ? cnt[e] : 0;
+        const int flag = c > 0;
+        int ftot, ctot;
+        const int fpos = block_exscan256(flag, scan_tmp, ftot);
+        const int cpos = block_exscan256(c, scan_tmp, ctot);
+        if (e < E) {
+            if (flag) {
+                const int a = na_base + fpos;
+                int p = pair_base + cpos;
+                ws.active[a] = e;
+                ws.off[a] = p;
+                ws.act_of[e] = a;
+                for (int i = 0; i < T * k; ++i)
+                    if (idx[i] == e) {
+                        const int t = i / k, j = i % k;
+                        ws.pair_tok[p] = t;
+                        ws.pair_slot[p] = j;
+                        ws.tok_pair[t * (k + S) + j] = p;
+                        ++p;
+                    }
+            } else {
+                ws.act_of[e] = -1;
+            }
+        }
+        na_base += ftot;
+        pair_base += ctot;
+    }
+    for (int i = tid; i < S; i += 256) {
+        const int a = na_base + i;
+        ws.active[a] = E + i;
+        ws.off[a] = pair_base + i * T;
+        ws.act_of[E + i] = a;
+        for (int t = 0; t < T; ++t) {
+            const int p = pair_base + i * T + t;
+            ws.pair_tok[p] = t;
+            ws.pair_slot[p] = k + i;
+            ws.tok_pair[t * (k + S) + k + i] = p;
+        }
+    }
+    if (tid == 0) {
+        ws.off[na_base + S] = pair_base + S * T;
+        *ws.n_active = na_base + S;
+    }
+}
+
+// Router for few tokens (T <= NT), one kernel: CTA e computes the fp64 logit
+// of expert e for every token, all CTAs share the Q8_0 of x (natural codes
+// and the records the expert kernels stage), and the last CTA to finish
+// selects every token's experts and builds the batch-union tables.
+// blockDim.x == 256; dynamic smem = select_smem_bytes(E, G) + 4*E.
+template <int NT, int BITS>
+__global__ void __launch_bounds__(256) k_router_small(
+    const float *__restrict__ x, int T, int H, const float *__restrict__ Wr,
+    const float *__restrict__ bias, int E, int S, int G, int gk, int k, float rsf, RouteWs ws,
+    uint8_t *__restrict__ xrec, int8_t *__restrict__ xq, float *__restrict__ xd,
+    int do_union, int32_t *__restrict__ idx_out, float *__restrict__ w_out) {
+    extern __shared__ __align__(16) uint8_t smem_r[];
+    __shared__ double red[8][NT];
+    __shared__ int is_last;
+    __shared__ int scan_tmp[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int e = blockIdx.x;
+    // ---- logit of expert e for every token (fp64 sum of exact products)
+    {
+        double acc[NT];
+#pragma unroll
+        for (int t = 0; t < NT; ++t) acc[t] = 0.0;
+        const float4 *w4 = reinterpret_cast<const float4 *>(Wr + (int64_t)e * H);
+        for (int i = tid; i < H / 4; i += 256) {
+            const float4 wv = __ldg(w4 + i);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                if (t < T) {
+                    const float4 xv = __ldg(reinterpret_cast<const float4 *>(x + (int64_t)t * H) + i);
+                    acc[t] = fma((double)xv.x, (double)wv.x, acc[t]);
+                    acc[t] = fma((double)xv.y, (double)wv.y, acc[t]);
+                    acc[t] = fma((double)xv.z, (double)wv.z, acc[t]);
+                    acc[t] = fma((double)xv.w, (double)wv.w, acc[t]);
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            const double v = warp_sum(acc[t]);
+            if (lane == 0) red[warp][t] = v;
+        }
+        __syncthreads();
+        if (tid < T) {
+            double l = 0.0;
+            for (int w = 0; w < 8; ++w) l += red[w][tid];
+            const double sg = 1.0 / (1.0 + exp(-l));
+            ws.s[(int64_t)tid * E + e] = sg;
+            ws.c[(int64_t)tid * E + e] = sg + (double)bias[e];
+        }
+    }
+    // ---- Q8_0(x): warps of all CTAs share the T * H/32 blocks
+    if (do_union) {
+        const int nb = H / COLI_QBLK;
+        const int rb = rec_bytes(H);
+        for (int blk = blockIdx.x * 8 + warp; blk < T * nb; blk += gridDim.x * 8) {
+            const int t = blk / nb, b = blk % nb;
+            const float v = __ldg(x + (int64_t)t * H + b * COLI_QBLK + lane);
+            q8_block_to_record<BITS>(v, b, H, xrec + (size_t)t * rb, xq + (int64_t)t * H,
+                                     xd + (int64_t)t * nb);
+        }
+    }
+    // ---- last CTA: selection and the union tables
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) is_last = (atomicAdd(ws.counter, 1u) == (unsigned)(gridDim.x - 1));
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    const SelectSmem sm = carve_select(smem_r, E, G);
+    int32_t *idx_dst = do_union ? ws.idx : idx_out;
+    float *w_dst = do_union ? ws.w : w_out;
+    for (int t = 0; t < T; ++t)
+        cta_select_token(ws.c + (int64_t)t * E, ws.s + (int64_t)t * E, E, G, gk, k, rsf, sm,
+                         idx_dst + t * k, w_dst + t * k);
+    if (do_union) {
+        int *cnt = reinterpret_cast<int *>(smem_r + select_smem_bytes(E, G));
+        int *idx_s = cnt + E;
+        cta_union_small(ws, idx_dst, T, E, S, k, cnt, idx_s, scan_tmp);
+    }
+    __syncthreads();
+    if (tid == 0) *ws.counter = 0u;
+}
+
+// Q8_0 of x for many tokens: natural codes and scales plus the records.
+template <int BITS>
+__global__ void k_x_prep(const float *__restrict__ x, int T, int H, uint8_t *__restrict__ xrec,
+                         int8_t *__restrict__ xq, float *__restrict__ xd) {
+    const int lane = threadIdx.x & 31;
+    const int nb = H / COLI_QBLK, rb = rec_bytes(H);
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t blk = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+         blk < (int64_t)T * nb; blk += nwarps) {
+        const int t = (int)(blk / nb), b = (int)(blk % nb);
+        const float v = __ldg(x + (int64_t)t * H + b * COLI_QBLK + lane);
+        q8_block_to_record<BITS>(v, b, H, xrec + (size_t)t * rb, xq + (int64_t)t * H,
+                                 xd + (int64_t)t * nb);
+    }
 }
 
 }  // namespace coli

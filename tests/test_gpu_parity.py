@@ -176,6 +176,20 @@ def test_invalid_arguments_are_rejected():
     gl.close()
 
 
+def test_bounded_wait_reports_timeout_and_handle_recovers():
+    """A device wait that nothing satisfies gives up after about a second and
+    is reported as COLI_ETIMEOUT; the handle keeps working afterwards."""
+    cfg = _small_cfg(seed=10)
+    gl = GpuLayer(cfg, max_tokens=4)
+    assert gl.handle.device_status() == qe.COLI_OK
+    gl.handle.dbg_wait_probe()
+    assert gl.handle.device_status() == qe.COLI_ETIMEOUT
+    assert gl.handle.device_status() == qe.COLI_OK
+    compare_forward(gl, synth.tokens(cfg, T=4, device=DEV))
+    assert gl.handle.device_status() == qe.COLI_OK
+    gl.close()
+
+
 # ------------------------------------------------------- full-size workloads
 @pytest.fixture(scope="module")
 def glm52_layer():
