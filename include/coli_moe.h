@@ -200,6 +200,34 @@ coli_status coli_dbg_block_sums(const void *codes, int wfmt, int64_t rows, int64
 coli_status coli_dbg_last_forward(coli_moe *m, int T, int32_t *idx, float *w, int8_t *hq,
                                   float *hd, coli_stream_t stream);
 
+/* Routing that allocates nothing (no counterpart on the pages; the pages'
+ * engine runs on the CPU and never faces this).  Same result as coli_router
+ * for the same inputs, but without a coli_moe handle: the router's scratch
+ * (fp64 sigmoid and choice scores and a completion ticket) lives in one
+ * fixed array inside the library instead of a workspace that
+ * coli_moe_create would cudaMalloc.  It is for callers that cannot allocate
+ * device memory at the point where they route: a process whose memory is
+ * already handed out to a caching allocator or a fixed budget, or a
+ * latency-critical loop that cannot take cudaMalloc's implicit
+ * synchronisation.  The call itself makes no cudaMalloc, cudaFree or other
+ * allocating call.
+ *   cfg:      layer shape (only hidden, n_routed, n_shared, top_k, n_group,
+ *             topk_group and routed_scaling_factor are used; the config must
+ *             still be valid as for coli_moe_create);
+ *   router_w [E][H], bias [E], x [T][H] fp32 device pointers;
+ *   idx [T][k] int32, w [T][k] fp32 device outputs, as coli_router.
+ * Limits: 1 <= T <= 8 tokens and n_routed <= 1024; larger requests return
+ * COLI_EINVAL.  The fixed array holds 131,328 bytes on every GPU that loads
+ * the library, until the process exits.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call on a device shares the one array
+ * and it keeps the last call's contents (the ticket is cleared at the start
+ * of each call): calls that overlap on the GPU, e.g. on two streams, race. */
+coli_status coli_router_static(const coli_moe_config *cfg, const float *router_w,
+                               const float *bias, const float *x, int T, int32_t *idx, float *w,
+                               coli_stream_t stream);
+
 /* Test hook for the bounded waits (no counterpart on the pages): one thread
  * waits on an mbarrier that nothing ever arrives at, through the same bounded
  * wait the pipelined kernels use.  The wait gives up after about one second

@@ -81,6 +81,7 @@ def lib():
         "coli_dbg_last_forward": ([vp, ci, vp, vp, vp, vp, vp], ci),
         "coli_dbg_wait_probe": ([vp, vp], ci),
         "coli_moe_device_status": ([vp, vp], ci),
+        "coli_router_static": ([vp, vp, vp, vp, ci, vp, vp, vp], ci),
     }
     for name, (args, res) in sigs.items():
         f = getattr(L, name)
@@ -142,6 +143,25 @@ def dbg_block_sums(codes, bits, K, xq, stream=None):
     _check(lib().coli_dbg_block_sums(_ptr(codes), bits, rows, K, _ptr(xq), T, _ptr(S),
                                      _stream(stream)))
     return S
+
+
+def _config(cfg, max_tokens=None):
+    return _Config(cfg["hidden"], cfg["inter"], cfg["n_routed"], cfg["n_shared"], cfg["top_k"],
+                   cfg["n_group"], cfg["topk_group"], cfg["routed_scaling_factor"], cfg["bits"],
+                   cfg.get("max_tokens", 1) if max_tokens is None else max_tokens)
+
+
+def router_static(cfg, router_w, bias, x, idx=None, w=None, stream=None):
+    """coli_router_static: routing without a handle and without any device
+    allocation inside the library (T <= 8, n_routed <= 1024)."""
+    T = x.shape[0]
+    k = cfg["top_k"]
+    idx = torch.empty((T, k), dtype=torch.int32, device=x.device) if idx is None else idx
+    w = torch.empty((T, k), dtype=torch.float32, device=x.device) if w is None else w
+    c = _config(cfg, max_tokens=max(T, 1))
+    _check(lib().coli_router_static(ctypes.byref(c), _ptr(router_w), _ptr(bias), _ptr(x), T,
+                                    _ptr(idx), _ptr(w), _stream(stream)))
+    return idx, w
 
 
 class Expert:

@@ -628,6 +628,36 @@ __global__ void k_gather_h(const int32_t *__restrict__ tok_pair, const int8_t *_
     }
 }
 
+// ---------------------------------------------------------------------------
+// Scratch of coli_router_static: fp64 sigmoid scores s [T][E] and choice
+// scores c [T][E] for at most ROUTER_STATIC_MAX_T tokens and
+// ROUTER_STATIC_MAX_E experts, then the last-CTA ticket.  A file-scope device
+// array: every GPU that loads the library holds it until the process exits,
+// and every coli_router_static call on that GPU shares it.
+constexpr int ROUTER_STATIC_MAX_T = 8;
+constexpr int ROUTER_STATIC_MAX_E = 1024;
+constexpr size_t ROUTER_STATIC_SC_BYTES = (size_t)ROUTER_STATIC_MAX_T * ROUTER_STATIC_MAX_E * 8;
+constexpr size_t ROUTER_STATIC_BYTES = 2 * ROUTER_STATIC_SC_BYTES + 256;
+static __device__ __align__(256) unsigned char g_router_scratch[ROUTER_STATIC_BYTES];
+
+// Device address of g_router_scratch per device, looked up once per device
+// with that device current.  In host code the symbol is only a stand-in.
+std::mutex g_router_scratch_mu;
+void *g_router_scratch_dev[128] = {nullptr};
+
+coli_status router_scratch_address(int dev, void **out) {
+    if (dev < 0 || dev >= 128) return fail(COLI_EUNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_router_scratch_mu);
+    if (!g_router_scratch_dev[dev]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_router_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(router scratch)");
+        g_router_scratch_dev[dev] = p;
+    }
+    *out = g_router_scratch_dev[dev];
+    return COLI_OK;
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -872,6 +902,50 @@ coli_status coli_moe_device_status(coli_moe *m, coli_stream_t stream) {
         return fail(COLI_ETIMEOUT, "a device-side wait gave up (error word %d)", word);
     }
     return COLI_OK;
+}
+
+coli_status coli_router_static(const coli_moe_config *cfg, const float *router_w,
+                               const float *bias, const float *x, int T, int32_t *idx, float *w,
+                               coli_stream_t stream) {
+    g_last_error.clear();
+    std::string why;
+    if (!cfg_valid(cfg, &why)) return fail(COLI_EINVAL, "invalid config: %s", why.c_str());
+    if (T < 1 || T > ROUTER_STATIC_MAX_T)
+        return fail(COLI_EINVAL, "coli_router_static takes 1 <= T <= %d tokens (got %d)",
+                    ROUTER_STATIC_MAX_T, T);
+    if (cfg->n_routed > ROUTER_STATIC_MAX_E)
+        return fail(COLI_EINVAL, "coli_router_static takes at most %d routed experts (got %d)",
+                    ROUTER_STATIC_MAX_E, cfg->n_routed);
+    if (!router_w || !bias || !x || !idx || !w) return fail(COLI_EINVAL, "null pointer");
+    if (!aligned16(router_w) || !aligned16(bias) || !aligned16(x) || !aligned16(idx) || !aligned16(w))
+        return fail(COLI_EINVAL, "pointers must be 16-byte aligned");
+    int dev = 0;
+    COLI_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    void *base = nullptr;
+    coli_status st = router_scratch_address(dev, &base);
+    if (st != COLI_OK) return st;
+    const int E = cfg->n_routed;
+    RouteWs rw{};
+    rw.s = (double *)base;
+    rw.c = (double *)((char *)base + ROUTER_STATIC_SC_BYTES);
+    rw.counter = (uint32_t *)((char *)base + 2 * ROUTER_STATIC_SC_BYTES);
+    cudaStream_t s = (cudaStream_t)stream;
+    // the ticket must start at zero; s and c are fully written before use
+    COLI_CUDA(cudaMemsetAsync(rw.counter, 0, sizeof(uint32_t), s), "clear router ticket");
+    const size_t smem = select_smem(*cfg) + 4 * (size_t)E + 4 * (size_t)T * cfg->top_k;
+    void (*kern)(const float *, int, int, const float *, const float *, int, int, int, int, int,
+                 float, RouteWs, uint8_t *, int8_t *, float *, int, int32_t *, float *);
+    if (T <= 1) kern = k_router_small<1, 4>;
+    else if (T <= 2) kern = k_router_small<2, 4>;
+    else if (T <= 4) kern = k_router_small<4, 4>;
+    else kern = k_router_small<8, 4>;
+    st = allow_smem(kern, smem);
+    if (st != COLI_OK) return st;
+    Launch L(nullptr, s, "router_static");
+    kern<<<E, 256, smem, s>>>(x, T, cfg->hidden, router_w, bias, E, cfg->n_shared, cfg->n_group,
+                              cfg->topk_group, cfg->top_k, cfg->routed_scaling_factor, rw, nullptr,
+                              nullptr, nullptr, 0, idx, w);
+    return L.done();
 }
 
 coli_status coli_dbg_wait_probe(coli_moe *m, coli_stream_t stream) {
