@@ -97,6 +97,7 @@ struct coli_moe {
     float *x_in = nullptr, *y_out = nullptr;
     uint8_t *xrec = nullptr, *hrec = nullptr;
     int *err = nullptr;
+    unsigned long long *gbar = nullptr;  // grid-barrier arrival counter of the decode kernel
     int last_T = 0;
     std::map<const void *, int> occ_cache;  // kernel -> CTAs per SM (attributes already set)
     // profiling
@@ -118,7 +119,7 @@ struct Layout {
 
 struct WsOffsets {
     size_t s, c, idx, w, bitmap, prefix, counter, n_active, active, off, act_of, pair_tok,
-        pair_slot, tok_pair, xq, xd, hq, hd, e_pairs, x_in, y_out, experts, xrec, hrec, err;
+        pair_slot, tok_pair, xq, xd, hq, hd, e_pairs, x_in, y_out, experts, xrec, hrec, err, gbar;
     size_t total;
 };
 
@@ -178,6 +179,7 @@ WsOffsets layout_of(const coli_moe_config &c) {
     o.xrec = L.add(T * (size_t)rec_bytes((int)H));
     o.hrec = L.add(P * (size_t)rec_bytes((int)I));
     o.err = L.add(4);
+    o.gbar = L.add(8);
     o.total = L.total;
     return o;
 }
@@ -368,6 +370,25 @@ cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// Cooperative launch: every CTA of the grid is resident at once (required by
+// the front kernel's grid barrier); the launch fails instead of running a
+// grid that does not fit.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_coop(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                        cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ---- few-token path sizing ------------------------------------------------
 constexpr int SMEM_BUDGET = 227 * 1024;
 
@@ -386,99 +407,25 @@ int ring_stages(size_t fixed, size_t stage) {
     return (int)std::min<size_t>((SMEM_BUDGET - fixed) / stage, PIPE_MAX_STAGES);
 }
 
-PipePlan plan_gateup(const coli_moe *m, int T) {
+PipePlan plan_decode(const coli_moe *m, int T) {
     const auto &c = m->cfg;
     PipePlan p;
-    const int RB = c.hidden * c.wfmt / 8;
-    const int R = pipe_rows_per_stage(RB);
-    const int slices = R >= PIPE_CONSUMERS ? 1 : PIPE_CONSUMERS / R;
-    p.amax = std::min(c.n_routed, T * c.top_k) + c.n_shared;
+    const GuGeom g = gu_geometry(c.hidden, c.wfmt);
+    p.grid = m->nsm;  // one CTA per SM, all co-resident
     p.pmax = T * (c.top_k + c.n_shared);
-    p.stage = (size_t)R * RB;
-    const size_t fixed = pipe_hdr_bytes() + align128((size_t)(2 * p.amax + 1 + p.pmax) * 4) +
-                         align128((size_t)T * rec_bytes(c.hidden)) +
-                         (size_t)2 * 2 * 32 * slices * PIPE_MAX_TOK * 8;
-    p.ns = ring_stages(fixed, p.stage);
-    p.smem = fixed + (size_t)p.ns * p.stage;
-    p.grid = std::max(1, std::min(m->nsm, p.amax * (c.inter / 32)));
-    return p;
-}
-
-PipePlan plan_down(const coli_moe *m, int T) {
-    const auto &c = m->cfg;
-    PipePlan p;
-    const int RB = c.inter * c.wfmt / 8;
-    p.grid = std::min(m->nsm, c.hidden);
     p.rows_cap = (c.hidden + p.grid - 1) / p.grid;
-    p.stage_rows = std::max(1, std::min(p.rows_cap, PIPE_STAGE_MAX / RB));
-    p.stage = (size_t)p.stage_rows * RB;
-    p.pmax = T * (c.top_k + c.n_shared);
-    const size_t fixed = pipe_hdr_bytes() + align128((size_t)p.pmax * rec_bytes(c.inter)) +
-                         (size_t)p.pmax * p.rows_cap * 4;
-    p.ns = ring_stages(fixed, p.stage);
-    p.smem = fixed + (size_t)p.ns * p.stage;
+    const int RBI = c.inter * c.wfmt / 8;
+    p.stage_rows = std::max(1, std::min(p.rows_cap, PIPE_STAGE_MAX / RBI));
+    const size_t fixed = decode_smem(T, c.hidden, c.inter, c.n_routed, c.n_shared, c.n_group,
+                                     c.top_k, p.pmax, g.slices, p.rows_cap, 0).total;
+    p.ns = ring_stages(fixed, PIPE_STAGE_MAX);
+    p.smem = fixed + (size_t)p.ns * PIPE_STAGE_MAX;
     return p;
 }
 
 bool small_path_ok(const coli_moe *m, int T) {
-    if (T > PIPE_MAX_TOK) return false;
-    return plan_gateup(m, T).ns >= 2 && plan_down(m, T).ns >= 2;
-}
-
-template <int BITS>
-coli_status launch_small_path(coli_moe *m, const float *x, int T, float *out, cudaStream_t s) {
-    const auto &c = m->cfg;
-    coli_status st;
-    {   // router + Q8_0(x) records + selection + union
-        const size_t smem = select_smem(c) + 4 * (size_t)c.n_routed + 4 * (size_t)T * c.top_k;
-        int occ = 1;
-        void (*kern)(const float *, int, int, const float *, const float *, int, int, int, int,
-                     int, float, RouteWs, uint8_t *, int8_t *, float *, int, int32_t *, float *);
-        if (T <= 1) kern = k_router_small<1, BITS>;
-        else if (T <= 2) kern = k_router_small<2, BITS>;
-        else if (T <= 4) kern = k_router_small<4, BITS>;
-        else kern = k_router_small<8, BITS>;
-        st = prepare(m, kern, 256, smem, &occ);
-        if (st != COLI_OK) return st;
-        Launch L(m, s, "router");
-        kern<<<c.n_routed, 256, smem, s>>>(x, T, c.hidden, m->router_w, m->bias, c.n_routed,
-                                           c.n_shared, c.n_group, c.topk_group, c.top_k,
-                                           c.routed_scaling_factor, m->rw, m->xrec, m->xq, m->xd,
-                                           1, m->rw.idx, m->rw.w);
-        st = L.done();
-        if (st != COLI_OK) return st;
-    }
-    {   // gate/up + SwiGLU + Q8_0(h)
-        const PipePlan p = plan_gateup(m, T);
-        auto kern = k_gateup_pipe<BITS>;
-        int occ = 1;
-        st = prepare(m, kern, PIPE_THREADS, p.smem, &occ);
-        if (st != COLI_OK) return st;
-        Launch L(m, s, "gateup_pipe");
-        cudaError_t e = launch_ex(kern, dim3(p.grid), dim3(PIPE_THREADS), p.smem, s, true, m->rw,
-                                  (const ExpertDev *)m->experts_dev, (const uint8_t *)m->xrec, T,
-                                  c.hidden, c.inter, p.ns, p.amax, p.pmax, m->hrec, m->hq, m->hd,
-                                  m->err);
-        if (e != cudaSuccess) return cuda_fail(e, "gateup_pipe launch");
-        st = L.done();
-        if (st != COLI_OK) return st;
-    }
-    {   // down + combine
-        const PipePlan p = plan_down(m, T);
-        auto kern = k_down_pipe<BITS>;
-        int occ = 1;
-        st = prepare(m, kern, PIPE_THREADS, p.smem, &occ);
-        if (st != COLI_OK) return st;
-        Launch L(m, s, "down_pipe");
-        cudaError_t e = launch_ex(kern, dim3(p.grid), dim3(PIPE_THREADS), p.smem, s, true, m->rw,
-                                  (const ExpertDev *)m->experts_dev, (const uint8_t *)m->hrec, T,
-                                  c.hidden, c.inter, c.top_k, c.n_shared, p.ns, p.stage_rows,
-                                  p.rows_cap, out, m->err);
-        if (e != cudaSuccess) return cuda_fail(e, "down_pipe launch");
-        st = L.done();
-        if (st != COLI_OK) return st;
-    }
-    return COLI_OK;
+    if (T > PIPE_MAX_TOK || m->cfg.hidden < m->nsm) return false;
+    return plan_decode(m, T).ns >= 3;
 }
 
 coli_status launch_route(coli_moe *m, const float *x, int T, int32_t *idx, float *w,
@@ -532,6 +479,49 @@ coli_status launch_route(coli_moe *m, const float *x, int T, int32_t *idx, float
                                             c.top_k, c.routed_scaling_factor, idx, w, do_union);
         return L.done();
     }
+}
+
+template <int BITS>
+coli_status launch_small_path(coli_moe *m, const float *x, int T, float *out, cudaStream_t s) {
+    const auto &c = m->cfg;
+    const PipePlan p = plan_decode(m, T);
+    auto kern = k_moe_decode<BITS>;
+    int occ = 1;
+    coli_status st = prepare(m, kern, DECODE_THREADS, p.smem, &occ);
+    if (st != COLI_OK) return st;
+    if (occ < 1) return fail(COLI_EUNSUPPORTED, "decode kernel does not fit on an SM");
+    DecodeArgs fa{};
+    fa.x = x;
+    fa.Wr = m->router_w;
+    fa.bias = m->bias;
+    fa.T = T;
+    fa.H = c.hidden;
+    fa.I = c.inter;
+    fa.E = c.n_routed;
+    fa.S = c.n_shared;
+    fa.G = c.n_group;
+    fa.gk = c.topk_group;
+    fa.k = c.top_k;
+    fa.rsf = c.routed_scaling_factor;
+    fa.ws = m->rw;
+    fa.experts = m->experts_dev;
+    fa.xrec = m->xrec;
+    fa.xq = m->xq;
+    fa.xd = m->xd;
+    fa.hrec = m->hrec;
+    fa.hq = m->hq;
+    fa.hd = m->hd;
+    fa.out = out;
+    fa.err = m->err;
+    fa.gbar = m->gbar;
+    fa.ns = p.ns;
+    fa.pmax = p.pmax;
+    fa.rows_cap = p.rows_cap;
+    fa.down_rows = p.stage_rows;
+    Launch L(m, s, "moe_decode");
+    cudaError_t e = launch_coop(kern, dim3(p.grid), dim3(DECODE_THREADS), p.smem, s, fa);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_decode launch");
+    return L.done();
 }
 
 coli_status quant_q8_launch(coli_moe *m, const float *x, int64_t rows, int64_t len, int8_t *q,
@@ -781,6 +771,7 @@ coli_status coli_moe_create(const coli_moe_config *cfg, const float *router_w, c
     m->xrec = (uint8_t *)(b + o.xrec);
     m->hrec = (uint8_t *)(b + o.hrec);
     m->err = (int *)(b + o.err);
+    m->gbar = (unsigned long long *)(b + o.gbar);
     e = cudaMemset(m->ws_base, 0, o.total);
     if (e == cudaSuccess)
         e = cudaMemcpy(m->experts_dev, host.data(), sizeof(ExpertDev) * n, cudaMemcpyHostToDevice);

@@ -57,6 +57,16 @@ __device__ __forceinline__ uint4 ldg_stream(const void *p) {
     return r;
 }
 
+// 16-byte shared-memory load through a 32-bit shared address (volatile, so
+// it stays ordered after the mbarrier wait that made the data visible).
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
 // ---------------------------------------------------------------------------
 // Activation staging.  A weight row of K elements is read as V = K*BITS/128
 // uint4 vectors.  For vector v the activation codes it multiplies are stored
@@ -92,6 +102,70 @@ template <int BITS> __device__ __forceinline__ int stage_src(int pos) {
     return word * 16 + byte * 4 + f;
 }
 
+// Raw dp4a sums of one 16-byte weight vector with its activation words.
+// Nibbles / crumbs are read as unsigned fields u = code XOR 8 (int4) or
+// code XOR 2 (int2), i.e. code + 8 / code + 2; the caller subtracts
+// 8 (2) * (sum of the block's activation codes).  (x & m) ^ c compiles to one
+// LOP3 per field word.
+__device__ __forceinline__ int dot_byte(const uint4 w, const uint4 a) {
+    int s = dp4a_ss((int)w.x, (int)a.x, 0);
+    s = dp4a_ss((int)w.y, (int)a.y, s);
+    s = dp4a_ss((int)w.z, (int)a.z, s);
+    return dp4a_ss((int)w.w, (int)a.w, s);
+}
+__device__ __forceinline__ int dot_nib(const uint4 w, const uint4 a0, const uint4 a1) {
+    const unsigned M = 0x0F0F0F0Fu, C = 0x08080808u;
+    int s = dp4a_us((w.x & M) ^ C, (int)a0.x, 0);
+    s = dp4a_us(((w.x >> 4) & M) ^ C, (int)a0.y, s);
+    s = dp4a_us((w.y & M) ^ C, (int)a0.z, s);
+    s = dp4a_us(((w.y >> 4) & M) ^ C, (int)a0.w, s);
+    s = dp4a_us((w.z & M) ^ C, (int)a1.x, s);
+    s = dp4a_us(((w.z >> 4) & M) ^ C, (int)a1.y, s);
+    s = dp4a_us((w.w & M) ^ C, (int)a1.z, s);
+    return dp4a_us(((w.w >> 4) & M) ^ C, (int)a1.w, s);
+}
+__device__ __forceinline__ int dot_crumb2(unsigned w0, unsigned w1, const uint4 a0, const uint4 a1) {
+    const unsigned M = 0x03030303u, C = 0x02020202u;
+    int s = dp4a_us((w0 & M) ^ C, (int)a0.x, 0);
+    s = dp4a_us(((w0 >> 2) & M) ^ C, (int)a0.y, s);
+    s = dp4a_us(((w0 >> 4) & M) ^ C, (int)a0.z, s);
+    s = dp4a_us(((w0 >> 6) & M) ^ C, (int)a0.w, s);
+    s = dp4a_us((w1 & M) ^ C, (int)a1.x, s);
+    s = dp4a_us(((w1 >> 2) & M) ^ C, (int)a1.y, s);
+    s = dp4a_us(((w1 >> 4) & M) ^ C, (int)a1.z, s);
+    return dp4a_us(((w1 >> 6) & M) ^ C, (int)a1.w, s);
+}
+
+// Sum over the 32 lanes of U per-lane values at once (U = 1, 2 or 4): after
+// the call the total of value r is in every lane whose bits 4..(5-log2 U)
+// spell r (lane >> 4 for U = 2, lane >> 3 for U = 4).  Exchanges halves first,
+// so U values cost log2(U) + (5 - log2(U)) shuffle steps instead of 5 * U.
+template <int U>
+__device__ __forceinline__ double warp_sum_rows(const double (&v)[U]) {
+    const int lane = threadIdx.x & 31;
+    if (U == 1) return warp_sum(v[0]);
+    if (U == 2) {
+        const bool hi = lane & 16;
+        double keep = hi ? v[1] : v[0], give = hi ? v[0] : v[1];
+        keep += __shfl_xor_sync(0xffffffffu, give, 16);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) keep += __shfl_xor_sync(0xffffffffu, keep, o);
+        return keep;
+    }
+    // U == 4
+    const bool b4 = lane & 16, b3 = lane & 8;
+    double p0 = b4 ? v[2] : v[0], p1 = b4 ? v[3] : v[1];
+    const double g0 = b4 ? v[0] : v[2], g1 = b4 ? v[1] : v[3];
+    p0 += __shfl_xor_sync(0xffffffffu, g0, 16);
+    p1 += __shfl_xor_sync(0xffffffffu, g1, 16);
+    double keep = b3 ? p1 : p0;
+    const double give = b3 ? p0 : p1;
+    keep += __shfl_xor_sync(0xffffffffu, give, 8);
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) keep += __shfl_xor_sync(0xffffffffu, keep, o);
+    return keep;
+}
+
 // Integer partial dot of one weight vector with its staged activations.
 // Returns the raw dp4a sums for each 32-block fragment the vector covers
 // (one for BITS 8 -- half a block -- and 4, two for BITS 2), before the
@@ -99,52 +173,16 @@ template <int BITS> __device__ __forceinline__ int stage_src(int pos) {
 template <int BITS>
 __device__ __forceinline__ void vec_dot(const uint4 w, const uint4 *act, int V, int &s0, int &s1) {
     if (BITS == 8) {
-        uint4 a = act[0];
-        int s = 0;
-        s = dp4a_ss((int)w.x, (int)a.x, s);
-        s = dp4a_ss((int)w.y, (int)a.y, s);
-        s = dp4a_ss((int)w.z, (int)a.z, s);
-        s = dp4a_ss((int)w.w, (int)a.w, s);
-        s0 = s;
+        s0 = dot_byte(w, act[0]);
         s1 = 0;
     } else if (BITS == 4) {
         uint4 a0 = act[0], a1 = act[V];
-        unsigned t0 = w.x ^ 0x88888888u, t1 = w.y ^ 0x88888888u;
-        unsigned t2 = w.z ^ 0x88888888u, t3 = w.w ^ 0x88888888u;
-        int s = 0;
-        s = dp4a_us(t0 & 0x0F0F0F0Fu, (int)a0.x, s);
-        s = dp4a_us((t0 >> 4) & 0x0F0F0F0Fu, (int)a0.y, s);
-        s = dp4a_us(t1 & 0x0F0F0F0Fu, (int)a0.z, s);
-        s = dp4a_us((t1 >> 4) & 0x0F0F0F0Fu, (int)a0.w, s);
-        s = dp4a_us(t2 & 0x0F0F0F0Fu, (int)a1.x, s);
-        s = dp4a_us((t2 >> 4) & 0x0F0F0F0Fu, (int)a1.y, s);
-        s = dp4a_us(t3 & 0x0F0F0F0Fu, (int)a1.z, s);
-        s = dp4a_us((t3 >> 4) & 0x0F0F0F0Fu, (int)a1.w, s);
-        s0 = s;
+        s0 = dot_nib(w, a0, a1);
         s1 = 0;
     } else {
         uint4 a0 = act[0], a1 = act[V], a2 = act[2 * V], a3 = act[3 * V];
-        unsigned t0 = w.x ^ 0xAAAAAAAAu, t1 = w.y ^ 0xAAAAAAAAu;
-        unsigned t2 = w.z ^ 0xAAAAAAAAu, t3 = w.w ^ 0xAAAAAAAAu;
-        int s = 0, u = 0;
-        s = dp4a_us(t0 & 0x03030303u, (int)a0.x, s);
-        s = dp4a_us((t0 >> 2) & 0x03030303u, (int)a0.y, s);
-        s = dp4a_us((t0 >> 4) & 0x03030303u, (int)a0.z, s);
-        s = dp4a_us((t0 >> 6) & 0x03030303u, (int)a0.w, s);
-        s = dp4a_us(t1 & 0x03030303u, (int)a1.x, s);
-        s = dp4a_us((t1 >> 2) & 0x03030303u, (int)a1.y, s);
-        s = dp4a_us((t1 >> 4) & 0x03030303u, (int)a1.z, s);
-        s = dp4a_us((t1 >> 6) & 0x03030303u, (int)a1.w, s);
-        u = dp4a_us(t2 & 0x03030303u, (int)a2.x, u);
-        u = dp4a_us((t2 >> 2) & 0x03030303u, (int)a2.y, u);
-        u = dp4a_us((t2 >> 4) & 0x03030303u, (int)a2.z, u);
-        u = dp4a_us((t2 >> 6) & 0x03030303u, (int)a2.w, u);
-        u = dp4a_us(t3 & 0x03030303u, (int)a3.x, u);
-        u = dp4a_us((t3 >> 2) & 0x03030303u, (int)a3.y, u);
-        u = dp4a_us((t3 >> 4) & 0x03030303u, (int)a3.z, u);
-        u = dp4a_us((t3 >> 6) & 0x03030303u, (int)a3.w, u);
-        s0 = s;
-        s1 = u;
+        s0 = dot_crumb2(w.x, w.y, a0, a1);
+        s1 = dot_crumb2(w.z, w.w, a2, a3);
     }
 }
 
@@ -263,8 +301,11 @@ __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// Named barrier among `nthreads` threads (a multiple of 32), id 1..15.
+// Named barrier among `nthreads` threads (a multiple of 32), id 1..15.  The
+// warp reconverges first: bar.sync needs every thread of a warp to arrive at
+// the same instruction.
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
+    __syncwarp();
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 

@@ -391,13 +391,16 @@ __global__ void __launch_bounds__(256) k_down_combine(RouteWs ws,
 // ===========================================================================
 // Few-token (decode / verification) kernels: weight rows stream through a
 // shared-memory ring with cp.async.bulk copies issued by one producer thread
-// and completed on mbarriers; sixteen consumer warps run the integer dots out
-// of shared memory.  One CTA per SM, persistent.  Every wait is bounded: on a
+// and completed on mbarriers; eight consumer warps run the integer dots out
+// of shared memory (nine warps in all, so no SM sub-partition holds more than
+// three and each thread may use up to 168 registers).  One CTA per SM, persistent.  Every wait is bounded: on a
 // timeout the kernel records COLI_ETIMEOUT in *err, drains its own copies and
 // returns.
-constexpr int PIPE_CONSUMERS = 16;
+constexpr int PIPE_CONSUMERS = 8;
 constexpr int PIPE_THREADS = 32 * (PIPE_CONSUMERS + 1);
-constexpr int PIPE_STAGE_MAX = 48 * 1024;  // bytes of weights per ring stage (at most)
+// the decode kernel adds an epilogue warp: 8 consumers, producer, epilogue
+constexpr int DECODE_THREADS = 32 * (PIPE_CONSUMERS + 2);
+constexpr int PIPE_STAGE_MAX = 24 * 1024;  // bytes of weights per ring stage (at most)
 constexpr int PIPE_MAX_STAGES = 8;
 constexpr int PIPE_MAX_TOK = 8;            // tokens per expert on the few-token path
 constexpr int PIPE_PASS_TOK = 4;           // tokens per pass over a staged weight row
@@ -409,10 +412,10 @@ struct PipeBars {
     int abort;
 };
 
-__host__ __device__ inline size_t pipe_hdr_bytes() { return (sizeof(PipeBars) + 127) & ~(size_t)127; }
+__host__ __device__ inline size_t pipe_hdr_bytes() { return (sizeof(PipeBars) + 8 + 32 + 127) & ~(size_t)127; }
 __host__ __device__ inline size_t align128(size_t x) { return (x + 127) & ~(size_t)127; }
 
-// Gate/up rows per stage: a power of two dividing 32 with R * rowbytes <= 48 KB.
+// Gate/up rows per stage: a power of two dividing 32 with R * rowbytes <= 24 KB.
 __host__ __device__ inline int pipe_rows_per_stage(int rowbytes) {
     int r = 32;
     while (r > 1 && r * rowbytes > PIPE_STAGE_MAX) r >>= 1;
@@ -462,167 +465,188 @@ __device__ __forceinline__ void slice_dot(const uint4 *__restrict__ wrow, int v_
     }
 }
 
+// Gate/up stage geometry.  A stage holds R consecutive rows of one matrix;
+// each row is split into `slices` vector ranges; the R * slices units are
+// spread over the consumer warps, U per warp: warp w takes slice w % slices
+// of rows w / slices + k * (PIPE_CONSUMERS / slices), k < U.  When a row has
+// V = 96 * slices vectors with slices in {1, 2, 4} (hidden 6144 in every
+// format: int2 1, int4 2, int8 4) every lane owns exactly 3 vectors of its
+// slice (the register-resident single-token path: 16 units per 24 KB stage,
+// U = 2).
+struct GuGeom {
+    int R, slices, U;
+    bool fast;
+};
+__host__ __device__ inline GuGeom gu_geometry(int H, int bits) {
+    const int V = H * bits / 128, RB = H * bits / 8;
+    GuGeom g;
+    if (V % 96 == 0 && (V / 96 == 1 || V / 96 == 2 || V / 96 == 4)) {
+        g.slices = V / 96;
+        g.R = 16 / g.slices;
+        g.U = 16 / PIPE_CONSUMERS;
+        g.fast = true;
+    } else {
+        g.R = pipe_rows_per_stage(RB);
+        g.slices = g.R >= PIPE_CONSUMERS ? 1 : PIPE_CONSUMERS / g.R;
+        g.U = g.R * g.slices / PIPE_CONSUMERS;
+        g.fast = false;
+    }
+    return g;
+}
+
+// Activation of one token for the vectors a lane owns (VPL of them, lane +
+// 32 j past `vbase`), held in registers: codes, the block scales as fp64 and
+// the unsigned-offset correction  -off * sum_b xs_b * d_b  of those blocks.
+template <int BITS, int VPL> struct LaneAct {
+    static constexpr int PL = Fmt<BITS>::PLANES;
+    static constexpr int NBV = BITS == 2 ? 2 : 1;  // scales per vector
+    uint4 a[VPL][PL];
+    double d[VPL][NBV];
+    double corr;
+    __device__ __forceinline__ void load(const uint8_t *rec, int K, int V, int vbase) {
+        const int lane = threadIdx.x & 31;
+        const int nb = K / COLI_QBLK;
+        const int *xs = reinterpret_cast<const int *>(rec + K);
+        const float *xd = reinterpret_cast<const float *>(rec + K + 4 * nb);
+        corr = 0.0;
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+            const int v = vbase + lane + 32 * j;
+#pragma unroll
+            for (int p = 0; p < PL; ++p) a[j][p] = reinterpret_cast<const uint4 *>(rec)[p * V + v];
+            if (BITS == 8) {
+                d[j][0] = (double)xd[v >> 1];
+            } else if (BITS == 4) {
+                d[j][0] = (double)xd[v];
+                corr = fma(-8.0 * (double)xs[v], d[j][0], corr);
+            } else {
+                d[j][0] = (double)xd[2 * v];
+                d[j][1] = (double)xd[2 * v + 1];
+                corr = fma(-2.0 * (double)xs[2 * v], d[j][0], corr);
+                corr = fma(-2.0 * (double)xs[2 * v + 1], d[j][1], corr);
+            }
+        }
+    }
+    // lane partial of one weight row (its VPL vectors at wrow[vbase + lane + 32 j])
+    __device__ __forceinline__ double dot(const uint4 *wrow, int vbase) const {
+        const int lane = threadIdx.x & 31;
+        const uint32_t base = smem_u32(wrow + vbase + lane);
+        double acc = corr;
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+            const uint4 w = lds128(base + 512u * j);
+            if (BITS == 8) {
+                acc = fma((double)dot_byte(w, a[j][0]), d[j][0], acc);
+            } else if (BITS == 4) {
+                acc = fma((double)dot_nib(w, a[j][0], a[j][1]), d[j][0], acc);
+            } else {
+                acc = fma((double)dot_crumb2(w.x, w.y, a[j][0], a[j][1]), d[j][0], acc);
+                acc = fma((double)dot_crumb2(w.z, w.w, a[j][2], a[j][3]), d[j][1], acc);
+            }
+        }
+        return acc;
+    }
+};
+
 // Gate/up consumer work for one stage: row slices assigned to this warp,
 // NT tokens; writes the reduced sums to part[row][slice][token].
 template <int BITS, int NT>
-__device__ __forceinline__ void gateup_stage(const uint8_t *stage, int RB, int V, int H, int R,
-                                             int slices, int rows_per_warp, int row_base,
-                                             const uint8_t *acts, int rbH, const int *tok,
-                                             int i0, double *part_mat) {
+__device__ __forceinline__ void gateup_stage(const uint8_t *stage, int RB, int V, int H,
+                                             const GuGeom g, int row_base, const uint8_t *acts,
+                                             int rbH, const int *tok, int i0, double *part_mat,
+                                             int ntok) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint8_t *rec[NT];
 #pragma unroll
     for (int i = 0; i < NT; ++i) rec[i] = acts + (size_t)tok[i] * rbH;
-    for (int rr = 0; rr < rows_per_warp; ++rr) {
-        const int row = (slices == 1) ? warp * rows_per_warp + rr : warp / slices;
-        const int sl = (slices == 1) ? 0 : warp % slices;
-        const int v_lo = (int)((long long)sl * V / slices);
-        const int v_hi = (int)((long long)(sl + 1) * V / slices);
+    const int sl = warp % g.slices;
+    const int v_lo = (int)((long long)sl * V / g.slices);
+    const int v_hi = (int)((long long)(sl + 1) * V / g.slices);
+    for (int k = 0; k < g.U; ++k) {
+        const int row = warp / g.slices + k * (PIPE_CONSUMERS / g.slices);
         double acc[NT];
         slice_dot<BITS, NT>(reinterpret_cast<const uint4 *>(stage + (size_t)row * RB), v_lo, v_hi, V,
                             H, rec, acc);
 #pragma unroll
         for (int i = 0; i < NT; ++i) {
             const double tot = warp_sum(acc[i]);
-            if (lane == 0) part_mat[((row_base + row) * slices + sl) * PIPE_MAX_TOK + i0 + i] = tot;
+            if (lane == 0) part_mat[((row_base + row) * g.slices + sl) * ntok + i0 + i] = tot;
         }
     }
 }
 
-// Gate/up of the few-token path, fused with SwiGLU and Q8_0(h).
-// Items: (active expert, 32-row chunk of the intermediate); each item streams
-// the chunk's gate rows, then its up rows, R rows per stage.  The partial sums
-// of an item are double-buffered so the SwiGLU/Q8_0 epilogue of item n runs
-// while the next item's stages are consumed; one named barrier per item.
-// Dynamic smem: PipeBars | tables | T activation records | ring | partials.
+// Single-token fast path of one stage (geometry fast: U = 2 rows per warp,
+// 3 vectors per lane per row); activations already in registers.
+// Per-warp constants of the fast path: slice sl of rows r0 and r0 + rstep.
+struct FastGeo {
+    int sl, vbase, r0, rstep, slices;
+    __device__ __forceinline__ FastGeo(const GuGeom &g, int V) {
+        const int warp = threadIdx.x >> 5;
+        slices = g.slices;
+        sl = warp % g.slices;
+        vbase = sl * (V / g.slices);
+        rstep = PIPE_CONSUMERS / g.slices;
+        r0 = warp / g.slices;
+    }
+};
+
 template <int BITS>
-__global__ void __launch_bounds__(PIPE_THREADS, 1)
-    k_gateup_pipe(RouteWs ws, const ExpertDev *__restrict__ experts,
-                  const uint8_t *__restrict__ xrec, int T, int H, int I, int ns, int amax,
-                  int npairs_max, uint8_t *__restrict__ hrec, int8_t *__restrict__ hq, float *__restrict__ hd,
-                  int *__restrict__ err) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    PipeBars *bars = reinterpret_cast<PipeBars *>(smem);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int RB = H * BITS / 8;                 // bytes per weight row
-    const int V = H * BITS / 128;                // uint4 vectors per row
-    const int R = pipe_rows_per_stage(RB);       // rows per stage
-    const int spm = 32 / R;                      // stages per matrix per item
-    const int nchunk = I / 32;
-    const int rbH = rec_bytes(H);
-    const int slices = R >= PIPE_CONSUMERS ? 1 : PIPE_CONSUMERS / R;
-    const int rows_per_warp = R >= PIPE_CONSUMERS ? R / PIPE_CONSUMERS : 1;
-    int *t_active = reinterpret_cast<int *>(smem + pipe_hdr_bytes());
-    int *t_off = t_active + amax;
-    int *t_tok = t_off + amax + 1;
-    uint8_t *acts = smem + pipe_hdr_bytes() + align128((size_t)(2 * amax + 1 + npairs_max) * 4);
-    uint8_t *ring = acts + align128((size_t)T * rbH);
-    const size_t stage_bytes = (size_t)R * RB;
-    double *part = reinterpret_cast<double *>(ring + (size_t)ns * stage_bytes);
-    const size_t part_mat = (size_t)32 * slices * PIPE_MAX_TOK;  // doubles per (buffer, matrix)
-    pipe_init(bars, ns);
-    pdl_wait();
-    const int n_active = *ws.n_active;
-    const int n_pairs = ws.off[n_active];
-    for (int i = tid; i < n_active; i += blockDim.x) t_active[i] = ws.active[i];
-    for (int i = tid; i <= n_active; i += blockDim.x) t_off[i] = ws.off[i];
-    for (int i = tid; i < n_pairs; i += blockDim.x) t_tok[i] = ws.pair_tok[i];
-    __syncthreads();
-    pdl_launch_dependents();
-    const int n_items = n_active * nchunk;
-    const int steps = 2 * spm;
-    if (warp == PIPE_CONSUMERS) {
-        if (lane != 0) return;
-        // ------------------------------ producer
-        mbar_expect_tx(&bars->act, (uint32_t)(T * rbH));
-        bulk_g2s(acts, xrec, (uint32_t)(T * rbH), &bars->act);
-        long long s = 0;
-        for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-            const int a = item / nchunk, c = item % nchunk;
-            const ExpertDev ex = experts[t_active[a]];
-            for (int ms = 0; ms < steps; ++ms, ++s) {
-                const int slot = (int)(s % ns);
-                if (s >= ns && !mbar_wait(&bars->empty[slot], (uint32_t)(((s / ns) - 1) & 1), err)) {
-                    pipe_drain(bars, ns, s, s - ns, err);
-                    mbar_wait(&bars->act, 0, err);
-                    return;
-                }
-                const QMatDev M = (ms < spm) ? ex.gate : ex.up;
-                const int row0 = c * 32 + (ms % spm) * R;
-                mbar_expect_tx(&bars->full[slot], (uint32_t)stage_bytes);
-                bulk_g2s(ring + (size_t)slot * stage_bytes, M.codes + (size_t)row0 * RB,
-                         (uint32_t)stage_bytes, &bars->full[slot]);
-            }
-        }
-        return;  // the consumers wait for every copy
+__device__ __forceinline__ void gateup_stage_fast(const uint8_t *stage, int RB, const FastGeo &f,
+                                                  int row_base, const LaneAct<BITS, 3> &act,
+                                                  double *part_mat, int ntok) {
+    const int lane = threadIdx.x & 31;
+    double acc[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+        acc[k] = act.dot(reinterpret_cast<const uint4 *>(stage + (size_t)(f.r0 + k * f.rstep) * RB),
+                         f.vbase);
+    const double tot = warp_sum_rows<2>(acc);
+    if ((lane & 15) == 0) {
+        const int row = f.r0 + (lane >> 4) * f.rstep;
+        part_mat[((row_base + row) * f.slices + f.sl) * ntok] = tot;
     }
-    // ---------------------------------- consumers
-    // A timed-out wait sets bars->abort; every consumer warp still passes each
-    // named barrier, and all of them leave together right after one.
-    volatile int *abort = &bars->abort;
-    bool ok = mbar_wait(&bars->act, 0, err);
-    if (!ok) *abort = 1;
-    long long s = 0;
-    int buf = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x, buf ^= 1) {
-        const int a = item / nchunk, c = item % nchunk;
-        const int p0 = t_off[a];
-        const int ne = min(t_off[a + 1] - p0, PIPE_MAX_TOK);
-        const int *tok = t_tok + p0;
-        // the epilogue warps fetch their row scales early
-        float sg = 0.0f, su = 0.0f;
-        const ExpertDev ex = experts[t_active[a]];
-        if (warp < ne) {
-            sg = __ldg(ex.gate.scales + c * 32 + lane);
-            su = __ldg(ex.up.scales + c * 32 + lane);
-        }
-        double *pbuf = part + (size_t)buf * 2 * part_mat;
-        for (int ms = 0; ms < steps && ok; ++ms, ++s) {
-            const int slot = (int)(s % ns);
-            if (!mbar_wait(&bars->full[slot], (uint32_t)((s / ns) & 1), err)) {
-                ok = false;
-                *abort = 1;
-                break;
-            }
-            const uint8_t *stage = ring + (size_t)slot * stage_bytes;
-            double *pm = pbuf + (ms < spm ? 0 : part_mat);
-            const int row_base = (ms % spm) * R;
-            // tokens in passes of at most PIPE_PASS_TOK over the staged rows
-            for (int i0 = 0; i0 < ne; i0 += PIPE_PASS_TOK) {
-                const int n = min(PIPE_PASS_TOK, ne - i0);
-                const int *tk = tok + i0;
-                switch (n) {
-                    case 1: gateup_stage<BITS, 1>(stage, RB, V, H, R, slices, rows_per_warp, row_base, acts, rbH, tk, i0, pm); break;
-                    case 2: gateup_stage<BITS, 2>(stage, RB, V, H, R, slices, rows_per_warp, row_base, acts, rbH, tk, i0, pm); break;
-                    case 3: gateup_stage<BITS, 3>(stage, RB, V, H, R, slices, rows_per_warp, row_base, acts, rbH, tk, i0, pm); break;
-                    default: gateup_stage<BITS, 4>(stage, RB, V, H, R, slices, rows_per_warp, row_base, acts, rbH, tk, i0, pm); break;
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->empty[slot]);
-        }
-        named_bar(1, 32 * PIPE_CONSUMERS);
-        if (*abort) break;
-        // SwiGLU + Q8_0(h) of this item: warp i handles token i, lane = row in chunk
-        if (warp < ne) {
-            const int i = warp;
-            double ag = 0.0, au = 0.0;
-            for (int sl = 0; sl < slices; ++sl) {
-                ag += pbuf[((size_t)lane * slices + sl) * PIPE_MAX_TOK + i];
-                au += pbuf[part_mat + ((size_t)lane * slices + sl) * PIPE_MAX_TOK + i];
-            }
-            const float g = (float)(ag * (double)sg);
-            const float u = (float)(au * (double)su);
-            const double gd = (double)g;
-            const float h = (float)((gd / (1.0 + exp(-gd))) * (double)u);
-            const int p = p0 + i;
-            q8_block_to_record<BITS>(h, c, I, hrec + (size_t)p * rec_bytes(I), hq + (int64_t)p * I,
-                                     hd + (int64_t)p * (I / COLI_QBLK));
+}
+
+// 16-byte asynchronous global -> shared copies (L2 only), completed by
+// cp_async_wait_all.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Barrier across every CTA of a cooperative grid; called by one thread per
+// CTA between two CTA-level barriers.  `count` is a 64-bit arrival counter
+// that only grows: an arrival that returns v belongs to the generation ending
+// at (v / nblocks + 1) * nblocks, and the barrier opens when the counter gets
+// there (one atomic and, usually, one acquire load per CTA; no reset).
+// Bounded: false (and COLI_ETIMEOUT in *err) if the others did not arrive
+// within WAIT_LIMIT_CYCLES.
+__device__ inline bool grid_barrier(unsigned long long *count, unsigned nblocks, int *err) {
+    unsigned long long v;
+    asm volatile("atom.add.acq_rel.gpu.u64 %0, [%1], 1;" : "=l"(v) : "l"(count) : "memory");
+    const unsigned long long target = (v / nblocks + 1) * nblocks;
+    const long long t0 = clock64();
+    for (;;) {
+        unsigned long long now;
+        asm volatile("ld.acquire.gpu.u64 %0, [%1];" : "=l"(now) : "l"(count) : "memory");
+        if (now >= target) return true;
+        if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+            atomicExch(err, ERR_TIMEOUT);
+            return false;
         }
     }
 }
 
-// Down consumer work for one stage: rows w, w+16, ... of the stage, NT tokens
+// Down consumer work for one stage: rows w, w + 8, ... of the stage, NT tokens
 // starting at pair p; writes e = (float)(sum * row scale) to ebuf.
 template <int BITS, int NT>
 __device__ __forceinline__ void down_stage(const uint8_t *stage, int RB, int V, int I, int nr,
@@ -645,122 +669,594 @@ __device__ __forceinline__ void down_stage(const uint8_t *stage, int RB, int V, 
     }
 }
 
-// Down projection + combine of the few-token path.  CTA b owns a contiguous
-// range of output rows (balanced over the grid) and streams, for every active
-// expert in order, those rows of its down matrix; e values land in shared
-// memory and the CTA combines each token's slots in the fixed order (shared
-// experts first, then routed slots) in fp64.
-// Dynamic smem: PipeBars | all pairs' h records | ring | e values | row scales.
+// Down fast path for one pair: a warp's rows w + 8 k of the stage in groups
+// of four, activation of the pair in registers (VPL vectors per lane, full
+// rows).
+template <int BITS, int VPL>
+__device__ __forceinline__ void down_stage_fast(const uint8_t *stage, int RB, int V, int I, int nr,
+                                                const float *scales /* shared */, const uint8_t *rec,
+                                                int p, float *ebuf, int rows_cap, int row_off) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp >= nr) return;
+    LaneAct<BITS, VPL> act;
+    act.load(rec, I, V, 0);
+    for (int g0 = warp; g0 < nr; g0 += 4 * PIPE_CONSUMERS) {
+        double acc[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int row = g0 + PIPE_CONSUMERS * k;
+            acc[k] = (row < nr) ? act.dot(reinterpret_cast<const uint4 *>(stage + (size_t)row * RB), 0)
+                                : 0.0;
+        }
+        const double tot = warp_sum_rows<4>(acc);
+        if ((lane & 7) == 0) {
+            const int row = g0 + PIPE_CONSUMERS * (lane >> 3);
+            if (row < nr)
+                ebuf[(size_t)p * rows_cap + row_off + row] = (float)(tot * (double)scales[row]);
+        }
+    }
+}
+
+// ===========================================================================
+// The whole layer for few tokens in one persistent cooperative launch (one
+// CTA per SM, all co-resident).  One ring of weight stages runs through the
+// kernel: the shared experts' gate/up rows (issued while routing is still in
+// progress: they need none), the routed experts' gate/up rows, then the down
+// rows of this CTA's output-row range for every active expert (they need no
+// h, so they stream across the second grid barrier).
+//   P1  fp64 logits of experts b, b + grid, ...; Q8_0(x) records of a share
+//       of the blocks, to global memory.            -- grid barrier 1 --
+//   P2  every CTA copies the records, selects every token's experts and
+//       builds the batch-union tables in shared memory (CTA 0 publishes them).
+//   P3  gate/up items + SwiGLU + Q8_0(h) records, to global memory.
+//                                                   -- grid barrier 2 --
+//   P4  h records of every pair into shared memory; down rows of every active
+//       expert; fp64 combine of this CTA's rows, shared experts first.
+struct DecodeArgs {
+    const float *x;
+    const float *Wr;
+    const float *bias;
+    int T, H, I, E, S, G, gk, k;
+    float rsf;
+    RouteWs ws;
+    const ExpertDev *experts;
+    uint8_t *xrec;
+    int8_t *xq;
+    float *xd;
+    uint8_t *hrec;
+    int8_t *hq;
+    float *hd;
+    float *out;
+    int *err;
+    unsigned long long *gbar;   // grid-barrier arrival counter
+    int ns, pmax;
+    int rows_cap;       // output rows per CTA (max) in P4
+    int down_rows;      // down rows per stage
+};
+
+struct DecodeSmem {
+    size_t select, idxw, cnt, red, tables, act, ebuf, part, dscale, ring, total;
+};
+
+__host__ __device__ inline DecodeSmem decode_smem(int T, int H, int I, int E, int S, int G, int k,
+                                                  int pmax, int slices, int rows_cap, int ns) {
+    DecodeSmem d;
+    size_t o = pipe_hdr_bytes();
+    d.ring = o;
+    o += (size_t)ns * PIPE_STAGE_MAX;
+    d.select = o;
+    o += align128(select_smem_bytes(E, G));
+    d.idxw = o;
+    o += align128((size_t)T * k * 8);
+    d.cnt = o;
+    o += align128((size_t)E * 4);
+    d.red = o;
+    o += align128((size_t)2 * 8 * PIPE_MAX_TOK * 8);
+    d.tables = o;
+    o += align128((size_t)(3 * (E + S) + 1 + 3 * pmax + 4) * 4);
+    d.act = o;
+    const size_t xa = (size_t)T * rec_bytes(H), ha = (size_t)pmax * rec_bytes(I);
+    o += align128(xa > ha ? xa : ha);
+    d.ebuf = o;
+    o += align128((size_t)pmax * rows_cap * 4);
+    d.part = o;
+    const int ntok = T < PIPE_MAX_TOK ? T : PIPE_MAX_TOK;
+    o += align128((size_t)2 * 2 * 32 * slices * ntok * 8);
+    d.dscale = o;                         // down-row scales of this CTA, per active expert
+    const int amax = (E < T * k ? E : T * k) + S;
+    o += align128((size_t)amax * (rows_cap + 4) * 4);
+    d.total = o;
+    return d;
+}
+
+// Ring position: slot and phase parity advance together (no divisions).
+struct RingPos {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void next(int ns) {
+        if (++slot == ns) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+};
+
+// Stage cursor of one CTA: its gate/up items (j-th item, matrix step m), then
+// its down stages (active expert a, row sub-range sb).
+struct StageCursor {
+    int j = 0, m = 0, a = 0, sb = 0;
+    bool down = false;
+    __device__ __forceinline__ void next(int my_items, int steps, int subs) {
+        if (!down) {
+            if (++m == steps) {
+                m = 0;
+                if (++j >= my_items) {
+                    down = true;
+                    a = 0;
+                    sb = 0;
+                }
+            }
+        } else if (++sb == subs) {
+            sb = 0;
+            ++a;
+        }
+    }
+};
+
+struct EpiBars {
+    uint64_t part_full[2];   // the 8 consumer warps finished an item's partials
+    uint64_t part_free[2];   // the epilogue warp finished reading them
+};
+
 template <int BITS>
-__global__ void __launch_bounds__(PIPE_THREADS, 1)
-    k_down_pipe(RouteWs ws, const ExpertDev *__restrict__ experts,
-                const uint8_t *__restrict__ hrec, int T, int H, int I, int k, int S, int ns,
-                int stage_rows, int rows_cap, float *__restrict__ out, int *__restrict__ err) {
+__global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa) {
     extern __shared__ __align__(128) uint8_t smem[];
     PipeBars *bars = reinterpret_cast<PipeBars *>(smem);
-    const int rbI = rec_bytes(I);
-    const int n_pairs_max = T * (k + S);
-    const int RB = I * BITS / 8;
-    const int V = I * BITS / 128;
-    const size_t stage_bytes = (size_t)stage_rows * RB;
-    uint8_t *hacts = smem + pipe_hdr_bytes();
-    uint8_t *ring = hacts + align128((size_t)n_pairs_max * rbI);
-    float *ebuf = reinterpret_cast<float *>(ring + (size_t)ns * stage_bytes);  // [pairs][rows_cap]
+    EpiBars *ebars = reinterpret_cast<EpiBars *>(smem + sizeof(PipeBars) + 8);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int base = H / gridDim.x, rem = H % gridDim.x;
-    const int r0 = blockIdx.x * base + min((int)blockIdx.x, rem);
-    const int nrows = base + ((int)blockIdx.x < rem ? 1 : 0);
+    const int T = fa.T, H = fa.H, I = fa.I, E = fa.E, S = fa.S, k = fa.k;
+    const int RB = H * BITS / 8, V = H * BITS / 128;
+    const int RBI = I * BITS / 8, VI = I * BITS / 128;
+    const GuGeom geo = gu_geometry(H, BITS);
+    const int R = geo.R, slices = geo.slices, spm = 32 / R, steps = 2 * spm;
+    const int nchunk = I / 32, rbH = rec_bytes(H), rbI = rec_bytes(I), nbH = H / COLI_QBLK;
+    const int ns = fa.ns, G = gridDim.x;
+    const DecodeSmem L = decode_smem(T, H, I, E, S, fa.G, k, fa.pmax, slices, fa.rows_cap, ns);
+    uint8_t *ring = smem + L.ring;
+    SelectSmem sm = carve_select(smem + L.select, E, fa.G);
+    int *idx_s = reinterpret_cast<int *>(smem + L.idxw);
+    float *w_s = reinterpret_cast<float *>(idx_s + T * k);
+    int *cnt = reinterpret_cast<int *>(smem + L.cnt);
+    double *red = reinterpret_cast<double *>(smem + L.red);
+    RouteWs lw = fa.ws;
+    lw.active = reinterpret_cast<int32_t *>(smem + L.tables);
+    lw.off = lw.active + (E + S);
+    lw.act_of = lw.off + (E + S + 1);
+    lw.pair_tok = lw.act_of + (E + S);
+    lw.pair_slot = lw.pair_tok + fa.pmax;
+    lw.tok_pair = lw.pair_slot + fa.pmax;
+    lw.n_active = lw.tok_pair + fa.pmax;
+    int *flags = lw.n_active + 1;
+    uint8_t *acts = smem + L.act;       // x records in P2/P3, h records in P4
+    float *ebuf = reinterpret_cast<float *>(smem + L.ebuf);
+    double *part = reinterpret_cast<double *>(smem + L.part);
+    float *dscale = reinterpret_cast<float *>(smem + L.dscale);   // [active][rows_cap + 4]
+    const int ntok = T < PIPE_MAX_TOK ? T : PIPE_MAX_TOK;
+    const size_t part_mat = (size_t)32 * slices * ntok;
+    const int rbase = H / G, rrem = H % G;
+    const int r0 = blockIdx.x * rbase + min((int)blockIdx.x, rrem);
+    const int nrows = rbase + ((int)blockIdx.x < rrem ? 1 : 0);
+    const int subs = (nrows + fa.down_rows - 1) / fa.down_rows;
+    const size_t gu_bytes = (size_t)R * RB;
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ebars->part_full[i], PIPE_CONSUMERS);
+            mbar_init(&ebars->part_free[i], 1);
+        }
+    }
     pipe_init(bars, ns);
     __syncthreads();
-    // The routing tables were complete before the gate/up kernel started, so
-    // the producer may stream down weights before the gate/up grid finishes;
-    // the h records are read only after pdl_wait.
-    const int n_active = *ws.n_active;
-    const int subs = (nrows + stage_rows - 1) / stage_rows;
+    volatile int *abort = &bars->abort;
+    const int n_shared_items = S * nchunk;
+    auto item_of = [&](int j) { return (int)blockIdx.x + j * G; };
+    auto item_expert_chunk = [&](int item, int n_active, int &a, int &e, int &c) {
+        if (item < n_shared_items) {
+            const int q = item / nchunk;
+            a = n_active - S + q;
+            e = E + q;
+            c = item - q * nchunk;
+        } else {
+            const int q = (item - n_shared_items) / nchunk;
+            a = q;
+            e = -1;  // looked up in the tables by the caller
+            c = item - n_shared_items - q * nchunk;
+        }
+    };
+
     if (warp == PIPE_CONSUMERS) {
+        // ------------------------------ producer (lane 0 issues)
+        StageCursor cur;
+        RingPos rp;
+        int issued = 0;
+        // let the router-weight loads enter the memory queues first
+        asm volatile("bar.sync 4, %0;" ::"r"(32 * (PIPE_CONSUMERS + 1)) : "memory");
+        while (lane == 0 && issued < ns && item_of(cur.j) < n_shared_items) {
+            const int item = item_of(cur.j);
+            const int q = item / nchunk;
+            const ExpertDev ex = fa.experts[E + q];
+            const QMatDev M = (cur.m < spm) ? ex.gate : ex.up;
+            const int row0 = (item - q * nchunk) * 32 + (cur.m % spm) * R;
+            mbar_expect_tx(&bars->full[rp.slot], (uint32_t)gu_bytes);
+            bulk_g2s(ring + (size_t)rp.slot * PIPE_STAGE_MAX, M.codes + (size_t)row0 * RB,
+                     (uint32_t)gu_bytes, &bars->full[rp.slot]);
+            ++issued;
+            rp.next(ns);
+            cur.next(1 << 30, steps, subs);
+        }
+        if (lane == 0)  // warm L2 with the shared experts' down rows of this CTA
+            for (int i = 0; i < S; ++i)
+                bulk_prefetch_l2(fa.experts[E + i].down.codes + (size_t)r0 * RBI, (uint32_t)(nrows * RBI));
+        __syncwarp();
+        named_bar(2, DECODE_THREADS);        // routing tables ready (or aborted)
         if (lane != 0) return;
-        long long s = 0;
-        bool act_issued = false;
-        auto issue_act = [&]() {
-            pdl_wait();
-            const int n_pairs = ws.off[n_active];
-            mbar_expect_tx(&bars->act, (uint32_t)(n_pairs * rbI));
-            bulk_g2s(hacts, hrec, (uint32_t)(n_pairs * rbI), &bars->act);
-            act_issued = true;
+        if (*abort) {
+            pipe_drain(bars, ns, issued, 0, fa.err);
+            return;
+        }
+        const int n_active = *lw.n_active;
+        const int n_items = n_active * nchunk;
+        const int my_items = n_items > (int)blockIdx.x ? (n_items - 1 - (int)blockIdx.x) / G + 1 : 0;
+        const int n_total = my_items * steps + n_active * subs;
+        if (cur.j >= my_items && !cur.down) {  // no gate/up work was pending
+            cur.down = true;
+            cur.a = 0;
+            cur.sb = 0;
+        }
+        auto desc = [&](const StageCursor &c, uint32_t &bytes) -> const uint8_t * {
+            if (!c.down) {
+                int a, e, ch;
+                item_expert_chunk(item_of(c.j), n_active, a, e, ch);
+                if (e < 0) e = lw.active[a];
+                const QMatDev M = (c.m < spm) ? fa.experts[e].gate : fa.experts[e].up;
+                bytes = (uint32_t)gu_bytes;
+                return M.codes + (size_t)(ch * 32 + (c.m % spm) * R) * RB;
+            }
+            const int rs = r0 + c.sb * fa.down_rows;
+            const int nr = min(fa.down_rows, r0 + nrows - rs);
+            bytes = (uint32_t)(nr * RBI);
+            return fa.experts[lw.active[c.a]].down.codes + (size_t)rs * RBI;
         };
-        for (int a = 0; a < n_active; ++a) {
-            const QMatDev M = experts[ws.active[a]].down;
-            for (int sb = 0; sb < subs; ++sb, ++s) {
-                const int slot = (int)(s % ns);
-                if (s >= ns) {
-                    // the ring is full: the consumers need the h records to free it
-                    if (!act_issued) issue_act();
-                    if (!mbar_wait(&bars->empty[slot], (uint32_t)(((s / ns) - 1) & 1), err)) {
-                        pipe_drain(bars, ns, s, s - ns, err);
-                        mbar_wait(&bars->act, 0, err);
-                        return;
-                    }
+        // lookahead cursor for the L2 prefetch, ns stages ahead
+        StageCursor ahead = cur;
+        for (int i = 0; i < ns; ++i) ahead.next(my_items, steps, subs);
+        for (int st = issued; st < n_total; ++st) {
+            if (st >= ns && !mbar_wait(&bars->empty[rp.slot], rp.phase ^ 1u, fa.err)) {
+                pipe_drain(bars, ns, st, st - ns, fa.err);
+                return;
+            }
+            uint32_t bytes;
+            const uint8_t *src = desc(cur, bytes);
+            mbar_expect_tx(&bars->full[rp.slot], bytes);
+            bulk_g2s(ring + (size_t)rp.slot * PIPE_STAGE_MAX, src, bytes, &bars->full[rp.slot]);
+            if (st + ns < n_total) {
+                uint32_t b2;
+                const uint8_t *s2 = desc(ahead, b2);
+                bulk_prefetch_l2(s2, b2);
+            }
+            rp.next(ns);
+            cur.next(my_items, steps, subs);
+            ahead.next(my_items, steps, subs);
+        }
+        return;  // the consumers wait for every copy
+    }
+
+    if (warp == PIPE_CONSUMERS + 1) {
+        // ------------------------------ epilogue warp: SwiGLU + Q8_0(h) of
+        // every item, off the consumers' critical path
+        named_bar(2, DECODE_THREADS);
+        bool ok = !*abort;
+        if (ok) {
+            const int n_active = *lw.n_active;
+            const int n_items = n_active * nchunk;
+            int n = 0;
+            for (int item = blockIdx.x; item < n_items && ok; item += G, ++n) {
+                const int buf = n & 1;
+                int a, e, c;
+                item_expert_chunk(item, n_active, a, e, c);
+                if (e < 0) e = lw.active[a];
+                const int p0 = lw.off[a];
+                const int ne = min(lw.off[a + 1] - p0, PIPE_MAX_TOK);
+                const ExpertDev ex = fa.experts[e];
+                const float sg = __ldg(ex.gate.scales + c * 32 + lane);
+                const float su = __ldg(ex.up.scales + c * 32 + lane);
+                if (!mbar_wait(&ebars->part_full[buf], (uint32_t)((n >> 1) & 1), fa.err)) {
+                    ok = false;
+                    *abort = 1;
+                    break;
                 }
-                const int rs = r0 + sb * stage_rows;
-                const int nr = min(stage_rows, r0 + nrows - rs);
-                mbar_expect_tx(&bars->full[slot], (uint32_t)(nr * RB));
-                bulk_g2s(ring + (size_t)slot * stage_bytes, M.codes + (size_t)rs * RB,
-                         (uint32_t)(nr * RB), &bars->full[slot]);
+                const double *pbuf = part + (size_t)buf * 2 * part_mat;
+                for (int i = 0; i < ne; ++i) {
+                    double ag = 0.0, au = 0.0;
+                    for (int sl = 0; sl < slices; ++sl) {
+                        ag += pbuf[((size_t)lane * slices + sl) * ntok + i];
+                        au += pbuf[part_mat + ((size_t)lane * slices + sl) * ntok + i];
+                    }
+                    const float g = (float)(ag * (double)sg);
+                    const float u = (float)(au * (double)su);
+                    const double gd = (double)g;
+                    const float h = (float)((gd / (1.0 + exp(-gd))) * (double)u);
+                    const int pr = p0 + i;
+                    q8_block_to_record<BITS>(h, c, I, fa.hrec + (size_t)pr * rbI,
+                                             fa.hq + (int64_t)pr * I, fa.hd + (int64_t)pr * (I / COLI_QBLK));
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ebars->part_free[buf]);
             }
         }
-        if (!act_issued) issue_act();
+        // let the consumers enter grid barrier 2 once every h record is written
+        __syncwarp();
+        asm volatile("bar.arrive 3, %0;" ::"r"(32 * (PIPE_CONSUMERS + 1)) : "memory");
         return;
     }
-    pdl_wait();
-    pdl_launch_dependents();
-    volatile int *abort = &bars->abort;
-    bool ok = mbar_wait(&bars->act, 0, err);
-    if (!ok) *abort = 1;
-    long long s = 0;
-    for (int a = 0; a < n_active && ok; ++a) {
-        const QMatDev M = experts[ws.active[a]].down;
-        const int p0 = ws.off[a], ne = ws.off[a + 1] - p0;
-        for (int sb = 0; sb < subs; ++sb, ++s) {
-            const int slot = (int)(s % ns);
-            if (!mbar_wait(&bars->full[slot], (uint32_t)((s / ns) & 1), err)) {
+
+    // ---------------------------------- consumers
+    // P1: logits of experts b, b + G, ... (two per pass, loads issued four
+    // iterations at a time) and a share of Q8_0(x).  Every consumer thread
+    // first requests its first router-weight lines into L2 and then, without
+    // condition, releases the producer (barrier 4), so those requests enter
+    // the memory queues ahead of the shared-expert bulk copies.
+    if ((int)blockIdx.x < E) {
+        const int e1 = (int)blockIdx.x + G;
+        for (int i = tid; i < H / 4 && i < 4 * 256; i += 256) {
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(fa.Wr + (int64_t)blockIdx.x * H + 4 * i));
+            if (e1 < E) asm volatile("prefetch.global.L2 [%0];" ::"l"(fa.Wr + (int64_t)e1 * H + 4 * i));
+        }
+    }
+    __syncwarp();
+    asm volatile("bar.arrive 4, %0;" ::"r"(32 * (PIPE_CONSUMERS + 1)) : "memory");
+    for (int e0 = blockIdx.x; e0 < E; e0 += 2 * G) {
+        const int e1 = e0 + G;
+        const bool two = e1 < E;
+        double acc[2][PIPE_MAX_TOK];
+#pragma unroll
+        for (int t = 0; t < PIPE_MAX_TOK; ++t) acc[0][t] = acc[1][t] = 0.0;
+        const float4 *w40 = reinterpret_cast<const float4 *>(fa.Wr + (int64_t)e0 * H);
+        const float4 *w41 = reinterpret_cast<const float4 *>(fa.Wr + (int64_t)(two ? e1 : e0) * H);
+        const int H4 = H / 4;
+        for (int i0 = tid; i0 < H4; i0 += 4 * 256) {
+            float4 wa[4], wb[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * 256;
+                wa[u] = (i < H4) ? __ldg(w40 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+                wb[u] = (i < H4) ? __ldg(w41 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+
+#pragma unroll
+            for (int t = 0; t < PIPE_MAX_TOK; ++t) {
+                if (t < T) {
+                    float4 xv[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = i0 + u * 256;
+                        xv[u] = (i < H4) ? __ldg(reinterpret_cast<const float4 *>(fa.x + (int64_t)t * H) + i)
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        acc[0][t] = fma((double)xv[u].x, (double)wa[u].x, acc[0][t]);
+                        acc[0][t] = fma((double)xv[u].y, (double)wa[u].y, acc[0][t]);
+                        acc[0][t] = fma((double)xv[u].z, (double)wa[u].z, acc[0][t]);
+                        acc[0][t] = fma((double)xv[u].w, (double)wa[u].w, acc[0][t]);
+                        acc[1][t] = fma((double)xv[u].x, (double)wb[u].x, acc[1][t]);
+                        acc[1][t] = fma((double)xv[u].y, (double)wb[u].y, acc[1][t]);
+                        acc[1][t] = fma((double)xv[u].z, (double)wb[u].z, acc[1][t]);
+                        acc[1][t] = fma((double)xv[u].w, (double)wb[u].w, acc[1][t]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < PIPE_MAX_TOK; ++t) {
+            if (t < T) {
+                const double v0 = warp_sum(acc[0][t]);
+                const double v1 = warp_sum(acc[1][t]);
+                if (lane == 0) {
+                    red[(0 * PIPE_CONSUMERS + warp) * PIPE_MAX_TOK + t] = v0;
+                    red[(1 * PIPE_CONSUMERS + warp) * PIPE_MAX_TOK + t] = v1;
+                }
+            }
+        }
+        named_bar(1, 256);
+        if (tid < 2 * T && (tid < T || two)) {
+            const int jj = tid / T, t = tid % T;
+            const int e = jj ? e1 : e0;
+            double l = 0.0;
+            for (int w = 0; w < PIPE_CONSUMERS; ++w) l += red[(jj * PIPE_CONSUMERS + w) * PIPE_MAX_TOK + t];
+            const double sg = 1.0 / (1.0 + exp(-l));
+            fa.ws.s[(int64_t)t * E + e] = sg;
+            fa.ws.c[(int64_t)t * E + e] = sg + (double)fa.bias[e];
+        }
+        named_bar(1, 256);
+    }
+    for (int blk = blockIdx.x * PIPE_CONSUMERS + warp; blk < T * nbH; blk += G * PIPE_CONSUMERS) {
+        const int t = blk / nbH, b = blk % nbH;
+        const float v = __ldg(fa.x + (int64_t)t * H + b * COLI_QBLK + lane);
+        q8_block_to_record<BITS>(v, b, H, fa.xrec + (size_t)t * rbH, fa.xq + (int64_t)t * H,
+                                 fa.xd + (int64_t)t * nbH);
+    }
+    named_bar(1, 256);
+    if (tid == 0) flags[0] = grid_barrier(fa.gbar, G, fa.err) ? 1 : 0;
+    named_bar(1, 256);
+    if (!flags[0]) {
+        *abort = 1;
+    } else {
+        // P2: x records (async, overlapping the selection), selection, union
+        for (int i = tid; i < T * rbH / 16; i += 256) cp_async16(acts + 16 * i, fa.xrec + 16 * i);
+        const bool pub = blockIdx.x == 0;
+        for (int t = 0; t < T; ++t) {
+            sm.w_smem = w_s + t * k;
+            cta_select_token<SyncConsumers>(fa.ws.c + (int64_t)t * E, fa.ws.s + (int64_t)t * E, E,
+                                            fa.G, fa.gk, k, fa.rsf, sm, pub ? fa.ws.idx + t * k : nullptr,
+                                            pub ? fa.ws.w + t * k : nullptr, idx_s + t * k);
+        }
+        cta_union_small<SyncConsumers>(lw, T, E, S, k, cnt, idx_s, reinterpret_cast<int *>(red));
+        cp_async_wait_all();
+        named_bar(1, 256);
+        if (pub) {
+            const int na = *lw.n_active, np = lw.off[na];
+            for (int i = tid; i < na; i += 256) fa.ws.active[i] = lw.active[i];
+            for (int i = tid; i <= na; i += 256) fa.ws.off[i] = lw.off[i];
+            for (int i = tid; i < E + S; i += 256) fa.ws.act_of[i] = lw.act_of[i];
+            for (int i = tid; i < np; i += 256) {
+                fa.ws.pair_tok[i] = lw.pair_tok[i];
+                fa.ws.pair_slot[i] = lw.pair_slot[i];
+                fa.ws.tok_pair[i] = lw.tok_pair[i];
+            }
+            if (tid == 0) *fa.ws.n_active = na;
+        }
+    }
+    named_bar(2, DECODE_THREADS);        // tables ready: release producer and epilogue warp
+    if (*abort) {
+        __syncwarp();
+        asm volatile("bar.sync 3, %0;" ::"r"(32 * (PIPE_CONSUMERS + 1)) : "memory");
+        return;
+    }
+
+    // P3: gate/up items; partials go to the epilogue warp through part_full /
+    // part_free (two buffers)
+    const FastGeo fgeo(geo, V);
+    const int n_active = *lw.n_active;
+    const int n_items = n_active * nchunk;
+    RingPos rp;
+    bool ok = true;
+    int n = 0;
+    for (int item = blockIdx.x; item < n_items && ok; item += G, ++n) {
+        const int buf = n & 1;
+        int a, e, c;
+        item_expert_chunk(item, n_active, a, e, c);
+        const int p0 = lw.off[a];
+        const int ne = min(lw.off[a + 1] - p0, PIPE_MAX_TOK);
+        const int *tok = lw.pair_tok + p0;
+        const bool fast = geo.fast && ne == 1;
+        LaneAct<BITS, 3> act;
+        if (fast) act.load(acts + (size_t)tok[0] * rbH, H, V, fgeo.vbase);
+        if (n >= 2 && !mbar_wait(&ebars->part_free[buf], (uint32_t)(((n >> 1) - 1) & 1), fa.err)) {
+            ok = false;
+            *abort = 1;
+            break;
+        }
+        double *pbuf = part + (size_t)buf * 2 * part_mat;
+        for (int ms = 0; ms < steps; ++ms) {
+            if (!mbar_wait(&bars->full[rp.slot], rp.phase, fa.err)) {
                 ok = false;
                 *abort = 1;
                 break;
             }
-            const int rs = r0 + sb * stage_rows;
-            const int nr = min(stage_rows, r0 + nrows - rs);
-            const uint8_t *stage = ring + (size_t)slot * stage_bytes;
-            for (int i0 = 0; i0 < ne; i0 += PIPE_PASS_TOK) {
-                const int n = min(PIPE_PASS_TOK, ne - i0);
-                const float *sc = M.scales + rs;
-                const int ro = rs - r0;
-                switch (n) {
-                    case 1: down_stage<BITS, 1>(stage, RB, V, I, nr, sc, hacts, rbI, p0 + i0, ebuf, rows_cap, ro); break;
-                    case 2: down_stage<BITS, 2>(stage, RB, V, I, nr, sc, hacts, rbI, p0 + i0, ebuf, rows_cap, ro); break;
-                    case 3: down_stage<BITS, 3>(stage, RB, V, I, nr, sc, hacts, rbI, p0 + i0, ebuf, rows_cap, ro); break;
-                    default: down_stage<BITS, 4>(stage, RB, V, I, nr, sc, hacts, rbI, p0 + i0, ebuf, rows_cap, ro); break;
+            const uint8_t *stage = ring + (size_t)rp.slot * PIPE_STAGE_MAX;
+            double *pm = pbuf + (ms < spm ? 0 : part_mat);
+            const int row_base = (ms < spm ? ms : ms - spm) * R;
+            if (fast) {
+                gateup_stage_fast<BITS>(stage, RB, fgeo, row_base, act, pm, ntok);
+            } else {
+                for (int i0 = 0; i0 < ne; i0 += PIPE_PASS_TOK) {
+                    const int nn = min(PIPE_PASS_TOK, ne - i0);
+                    const int *tk = tok + i0;
+                    switch (nn) {
+                        case 1: gateup_stage<BITS, 1>(stage, RB, V, H, geo, row_base, acts, rbH, tk, i0, pm, ntok); break;
+                        case 2: gateup_stage<BITS, 2>(stage, RB, V, H, geo, row_base, acts, rbH, tk, i0, pm, ntok); break;
+                        case 3: gateup_stage<BITS, 3>(stage, RB, V, H, geo, row_base, acts, rbH, tk, i0, pm, ntok); break;
+                        default: gateup_stage<BITS, 4>(stage, RB, V, H, geo, row_base, acts, rbH, tk, i0, pm, ntok); break;
+                    }
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->empty[slot]);
+            if (lane == 0) mbar_arrive(&bars->empty[rp.slot]);
+            rp.next(ns);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ebars->part_full[buf]);
+    }
+    // down-row scales of this CTA's rows for every active expert (they need
+    // no h): 4-byte async copies, waited for with the h records below
+    if (!*abort) {
+        const int ds = fa.rows_cap + 4;
+        for (int i = tid; i < n_active * nrows; i += 256) {
+            const int a = i / nrows, r = i % nrows;
+            const float *src = fa.experts[lw.active[a]].down.scales + r0 + r;
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dscale + a * ds + r)),
+                         "l"(src)
+                         : "memory");
         }
     }
-    named_bar(1, 32 * PIPE_CONSUMERS);
+    // grid barrier 2: every h record is written (the epilogue warp arrives on
+    // barrier 3 when its last record is out; the producer keeps streaming)
+    __syncwarp();
+    asm volatile("bar.sync 3, %0;" ::"r"(32 * (PIPE_CONSUMERS + 1)) : "memory");
+    if (tid == 0) flags[0] = (!*abort && grid_barrier(fa.gbar, G, fa.err)) ? 1 : 0;
+    named_bar(1, 256);
+    if (!flags[0]) {
+        *abort = 1;
+        return;
+    }
+    // P4: h records of every pair, down rows, combine
+    const int n_pairs = lw.off[n_active];
+    for (int i = tid; i < n_pairs * rbI / 16; i += 256) cp_async16(acts + 16 * i, fa.hrec + 16 * i);
+    cp_async_wait_all();
+    named_bar(1, 256);
+    const int vpl = (VI % 32 == 0) ? VI / 32 : 0;
+    for (int a = 0; a < n_active && ok; ++a) {
+        const int p0 = lw.off[a], ne = lw.off[a + 1] - p0;
+        for (int sb = 0; sb < subs; ++sb) {
+            if (!mbar_wait(&bars->full[rp.slot], rp.phase, fa.err)) {
+                ok = false;
+                *abort = 1;
+                break;
+            }
+            const int rs = r0 + sb * fa.down_rows;
+            const int nr = min(fa.down_rows, r0 + nrows - rs);
+            const uint8_t *stage = ring + (size_t)rp.slot * PIPE_STAGE_MAX;
+            const float *sc = dscale + a * (fa.rows_cap + 4) + (rs - r0);
+            const int ro = rs - r0;
+            if (vpl == 1 || vpl == 2 || vpl == 4) {
+                for (int i = 0; i < ne; ++i) {
+                    const uint8_t *rec = acts + (size_t)(p0 + i) * rbI;
+                    if (vpl == 1) down_stage_fast<BITS, 1>(stage, RBI, VI, I, nr, sc, rec, p0 + i, ebuf, fa.rows_cap, ro);
+                    else if (vpl == 2) down_stage_fast<BITS, 2>(stage, RBI, VI, I, nr, sc, rec, p0 + i, ebuf, fa.rows_cap, ro);
+                    else down_stage_fast<BITS, 4>(stage, RBI, VI, I, nr, sc, rec, p0 + i, ebuf, fa.rows_cap, ro);
+                }
+            } else {
+                for (int i0 = 0; i0 < ne; i0 += PIPE_PASS_TOK) {
+                    const int nn = min(PIPE_PASS_TOK, ne - i0);
+                    switch (nn) {
+                        case 1: down_stage<BITS, 1>(stage, RBI, VI, I, nr, sc, acts, rbI, p0 + i0, ebuf, fa.rows_cap, ro); break;
+                        case 2: down_stage<BITS, 2>(stage, RBI, VI, I, nr, sc, acts, rbI, p0 + i0, ebuf, fa.rows_cap, ro); break;
+                        case 3: down_stage<BITS, 3>(stage, RBI, VI, I, nr, sc, acts, rbI, p0 + i0, ebuf, fa.rows_cap, ro); break;
+                        default: down_stage<BITS, 4>(stage, RBI, VI, I, nr, sc, acts, rbI, p0 + i0, ebuf, fa.rows_cap, ro); break;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->empty[rp.slot]);
+            rp.next(ns);
+        }
+    }
+    named_bar(1, 256);
     if (*abort) return;
     const int slots = k + S;
-    for (int q = tid; q < T * nrows; q += 32 * PIPE_CONSUMERS) {
+    for (int q = tid; q < T * nrows; q += 256) {
         const int t = q / nrows, row = q % nrows;
         double acc = 0.0;
         for (int jj = 0; jj < slots; ++jj) {
             const int j = jj < S ? k + jj : jj - S;
-            const int p = ws.tok_pair[t * slots + j];
-            const double ev = (double)ebuf[(size_t)p * rows_cap + row];
+            const int p = lw.tok_pair[t * slots + j];
+            const double ev = (double)ebuf[(size_t)p * fa.rows_cap + row];
             if (j < k)
-                acc = fma((double)ws.w[t * k + j], ev, acc);
+                acc = fma((double)w_s[t * k + j], ev, acc);
             else
                 acc += ev;
         }
-        out[(int64_t)t * H + r0 + row] = (float)acc;
+        fa.out[(int64_t)t * H + r0 + row] = (float)acc;
     }
 }
 

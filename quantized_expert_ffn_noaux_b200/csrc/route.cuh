@@ -125,7 +125,21 @@ __global__ void __launch_bounds__(256) k_route_logits_tiled(
 }
 
 // ---------------------------------------------------------------------------
-// Block-wide exclusive scan of one int per thread (blockDim.x == 256).
+// Synchronisation of the 256 threads that run the routing helpers: the whole
+// CTA (SyncAll), or the eight consumer warps of a warp-specialised CTA whose
+// producer warp does not take part (SyncConsumers, named barrier 1).
+struct SyncAll {
+    __device__ static void sync() { __syncthreads(); }
+};
+struct SyncConsumers {
+    __device__ static void sync() {
+        __syncwarp();
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+    }
+};
+
+// Block-wide exclusive scan of one int per thread (256 participating threads).
+template <typename Sync = SyncAll>
 __device__ __forceinline__ int block_exscan256(int v, int *tmp /*[8]*/, int &total) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     int inc = v;
@@ -135,7 +149,7 @@ __device__ __forceinline__ int block_exscan256(int v, int *tmp /*[8]*/, int &tot
         if (lane >= o) inc += n;
     }
     if (lane == 31) tmp[wid] = inc;
-    __syncthreads();
+    Sync::sync();
     int base = 0, tot = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -143,7 +157,7 @@ __device__ __forceinline__ int block_exscan256(int v, int *tmp /*[8]*/, int &tot
         if (i < wid) base += t;
         tot += t;
     }
-    __syncthreads();
+    Sync::sync();
     total = tot;
     return base + inc - v;
 }
@@ -165,6 +179,7 @@ struct SelectSmem {
     int *cand;      // [E]
     int *ncand;     // [1]
     int *sel;       // [32]
+    float *w_smem;  // optional [k] copy of the weights (set by the caller)
 };
 
 __host__ __device__ inline size_t select_smem_bytes(int E, int G) {
@@ -183,20 +198,22 @@ __device__ inline SelectSmem carve_select(void *base, int E, int G) {
     m.keep = (int *)p;           p += (size_t)G * 4;
     m.ncand = (int *)p;          p += 4;
     m.sel = (int *)p;
+    m.w_smem = nullptr;
     return m;
 }
 
+template <typename Sync = SyncAll>
 __device__ void cta_select_token(const double *c_row, const double *s_row, int E, int G, int gk,
                                  int k, float rsf, const SelectSmem &sm, int32_t *idx_out,
-                                 float *w_out) {
-    const int tid = threadIdx.x, nthr = blockDim.x;
+                                 float *w_out, int *idx_smem = nullptr) {
+    const int tid = threadIdx.x, nthr = 256;
     const int per = E / G;
     for (int e = tid; e < E; e += nthr) {
         sm.c[e] = __ldcg(c_row + e);
         sm.s[e] = __ldcg(s_row + e);
     }
     if (tid == 0) *sm.ncand = 0;
-    __syncthreads();
+    Sync::sync();
     for (int e = tid; e < E; e += nthr) {
         const int g = e / per;
         const double v = sm.c[e];
@@ -210,12 +227,12 @@ __device__ void cta_select_token(const double *c_row, const double *s_row, int E
         if (r == 0) sm.top1[g] = v;
         if (r == 1) sm.top2[g] = v;
     }
-    __syncthreads();
+    Sync::sync();
     for (int g = tid; g < G; g += nthr) {
         const double v = sm.top1[g] + (per > 1 ? sm.top2[g] : 0.0);
         sm.top2[g] = v;  // reuse: group score
     }
-    __syncthreads();
+    Sync::sync();
     for (int g = tid; g < G; g += nthr) {
         const double v = sm.top2[g];
         int r = 0;
@@ -225,10 +242,10 @@ __device__ void cta_select_token(const double *c_row, const double *s_row, int E
         }
         sm.keep[g] = r < gk;
     }
-    __syncthreads();
+    Sync::sync();
     for (int e = tid; e < E; e += nthr)
         if (sm.keep[e / per] && sm.grank[e] < k) sm.cand[atomicAdd(sm.ncand, 1)] = e;
-    __syncthreads();
+    Sync::sync();
     const int n = *sm.ncand;
     for (int i = tid; i < n; i += nthr) {
         const int e = sm.cand[i];
@@ -241,17 +258,22 @@ __device__ void cta_select_token(const double *c_row, const double *s_row, int E
         }
         if (r < k) sm.sel[r] = e;
     }
-    __syncthreads();
+    Sync::sync();
     if (tid == 0) {
-        double ssum = 0.0;
+        double ssum = 0.0;  // slot order, as the weights' definition sums
         for (int j = 0; j < k; ++j) ssum += sm.s[sm.sel[j]];
-        for (int j = 0; j < k; ++j) {
-            const int e = sm.sel[j];
-            idx_out[j] = e;
-            w_out[j] = (float)((sm.s[e] / ssum) * (double)rsf);
-        }
+        sm.c[0] = ssum;     // c is no longer needed
     }
-    __syncthreads();
+    Sync::sync();
+    if (tid < k) {
+        const int e = sm.sel[tid];
+        const float wj = (float)((sm.s[e] / sm.c[0]) * (double)rsf);
+        if (idx_out) idx_out[tid] = e;
+        if (w_out) w_out[tid] = wj;
+        if (idx_smem) idx_smem[tid] = e;
+        if (sm.w_smem) sm.w_smem[tid] = wj;
+    }
+    Sync::sync();
 }
 
 // One CTA (256 threads) per token: cta_select_token.  With `do_union`, the
@@ -348,26 +370,25 @@ __global__ void __launch_bounds__(256) k_route_select(
 // Batch-union tables for few tokens (T * k <= 256), built by one CTA from
 // idx [T][k]: active experts ascending (shared experts last), each expert's
 // tokens in token order.
-__device__ void cta_union_small(RouteWs ws, const int32_t *idx_g, int T, int E, int S, int k,
-                                int *cnt /*smem [E]*/, int *idx /*smem [T*k]*/,
+template <typename Sync = SyncAll>
+__device__ void cta_union_small(RouteWs ws, int T, int E, int S, int k,
+                                int *cnt /*smem [E]*/, const int *idx /*smem [T*k]*/,
                                 int *scan_tmp /*smem [8]*/) {
     const int tid = threadIdx.x;
-    for (int i = tid; i < T * k; i += 256) idx[i] = idx_g[i];
-    __syncthreads();
     for (int e = tid; e < E; e += 256) {
         int c = 0;
         for (int i = 0; i < T * k; ++i) c += (idx[i] == e);
         cnt[e] = c;
     }
-    __syncthreads();
+    Sync::sync();
     int na_base = 0, pair_base = 0;
     for (int e0 = 0; e0 < E; e0 += 256) {
         const int e = e0 + tid;
         const int c = (e < E) ? cnt[e] : 0;
         const int flag = c > 0;
         int ftot, ctot;
-        const int fpos = block_exscan256(flag, scan_tmp, ftot);
-        const int cpos = block_exscan256(c, scan_tmp, ctot);
+        const int fpos = block_exscan256<Sync>(flag, scan_tmp, ftot);
+        const int cpos = block_exscan256<Sync>(c, scan_tmp, ctot);
         if (e < E) {
             if (flag) {
                 const int a = na_base + fpos;
@@ -479,14 +500,12 @@ __global__ void __launch_bounds__(256) k_router_small(
     const SelectSmem sm = carve_select(smem_r, E, G);
     int32_t *idx_dst = do_union ? ws.idx : idx_out;
     float *w_dst = do_union ? ws.w : w_out;
+    int *cnt = reinterpret_cast<int *>(smem_r + select_smem_bytes(E, G));
+    int *idx_s = cnt + E;
     for (int t = 0; t < T; ++t)
         cta_select_token(ws.c + (int64_t)t * E, ws.s + (int64_t)t * E, E, G, gk, k, rsf, sm,
-                         idx_dst + t * k, w_dst + t * k);
-    if (do_union) {
-        int *cnt = reinterpret_cast<int *>(smem_r + select_smem_bytes(E, G));
-        int *idx_s = cnt + E;
-        cta_union_small(ws, idx_dst, T, E, S, k, cnt, idx_s, scan_tmp);
-    }
+                         idx_dst + t * k, w_dst + t * k, idx_s + t * k);
+    if (do_union) cta_union_small(ws, T, E, S, k, cnt, idx_s, scan_tmp);
     __syncthreads();
     if (tid == 0) *ws.counter = 0u;
 }
