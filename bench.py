@@ -276,7 +276,13 @@ def run_coli(args, cfg, rank, world, device):
     avg_ms = ms_dom / n_dom
     prof_bytes = [bytes_per_step[s % L] for s in range(args.profile_steps)]
     frac_gu = gu_b / (gu_b + dn_b)
-    if dom.startswith("gateup"):
+    # router weights + bias (fp32) and the fp32 token rows read and written
+    router_b = cfg["n_routed"] * cfg["hidden"] * 4 + cfg["n_routed"] * 4
+    io_b = 2 * T * cfg["hidden"] * 4
+    if dom.startswith("moe_decode"):
+        # the whole layer in one launch: every union expert's three matrices
+        alg = statistics.mean(prof_bytes) + router_b + io_b
+    elif dom.startswith("gateup"):
         alg = statistics.mean(prof_bytes) * frac_gu
     elif dom.startswith("down"):
         alg = statistics.mean(prof_bytes) * (1 - frac_gu)

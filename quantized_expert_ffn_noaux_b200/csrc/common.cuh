@@ -136,34 +136,35 @@ __device__ __forceinline__ int dot_crumb2(unsigned w0, unsigned w1, const uint4 
     return dp4a_us(((w1 >> 6) & M) ^ C, (int)a1.w, s);
 }
 
-// Sum over the 32 lanes of U per-lane values at once (U = 1, 2 or 4): after
-// the call the total of value r is in every lane whose bits 4..(5-log2 U)
-// spell r (lane >> 4 for U = 2, lane >> 3 for U = 4).  Exchanges halves first,
-// so U values cost log2(U) + (5 - log2(U)) shuffle steps instead of 5 * U.
+// Sum over the 32 lanes of U per-lane values at once (U a power of two up to
+// 16): after the call the total of value r is in every lane with
+// lane >> (5 - log2 U) == r (lane >> 4 for U = 2, lane >> 3 for U = 4,
+// lane >> 2 for U = 8, lane >> 1 for U = 16).  Exchanging halves first costs
+// U - 1 + 5 - log2(U) shuffles instead of 5 U, on a chain 5 steps long.
 template <int U>
 __device__ __forceinline__ double warp_sum_rows(const double (&v)[U]) {
+    static_assert(U == 1 || U == 2 || U == 4 || U == 8 || U == 16, "U: power of two <= 16");
     const int lane = threadIdx.x & 31;
-    if (U == 1) return warp_sum(v[0]);
-    if (U == 2) {
-        const bool hi = lane & 16;
-        double keep = hi ? v[1] : v[0], give = hi ? v[0] : v[1];
-        keep += __shfl_xor_sync(0xffffffffu, give, 16);
+    double cur[U];
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1) keep += __shfl_xor_sync(0xffffffffu, keep, o);
-        return keep;
+    for (int i = 0; i < U; ++i) cur[i] = v[i];
+    // halving steps: lanes with the offset bit set keep the upper half of
+    // the values still in play and send the lower half, the others the
+    // reverse; after log2(U) steps value (lane >> (5 - log2 U)) is left
+#pragma unroll
+    for (int n = U, o = 16; n > 1; n >>= 1, o >>= 1) {
+        const bool hi = lane & o;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const double keep = hi ? cur[n / 2 + i] : cur[i];
+            const double give = hi ? cur[i] : cur[n / 2 + i];
+            cur[i] = keep + __shfl_xor_sync(0xffffffffu, give, o);
+        }
     }
-    // U == 4
-    const bool b4 = lane & 16, b3 = lane & 8;
-    double p0 = b4 ? v[2] : v[0], p1 = b4 ? v[3] : v[1];
-    const double g0 = b4 ? v[0] : v[2], g1 = b4 ? v[1] : v[3];
-    p0 += __shfl_xor_sync(0xffffffffu, g0, 16);
-    p1 += __shfl_xor_sync(0xffffffffu, g1, 16);
-    double keep = b3 ? p1 : p0;
-    const double give = b3 ? p0 : p1;
-    keep += __shfl_xor_sync(0xffffffffu, give, 8);
+    double r = cur[0];
 #pragma unroll
-    for (int o = 4; o > 0; o >>= 1) keep += __shfl_xor_sync(0xffffffffu, keep, o);
-    return keep;
+    for (int o = 32 / U / 2; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+    return r;
 }
 
 // Integer partial dot of one weight vector with its staged activations.
@@ -266,6 +267,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Bounded wait that yields the issue slots while it waits: for threads whose
+// wait is long and whose wake-up latency matters little (the producer thread
+// waiting for a free ring slot, the epilogue warp waiting for partials), so
+// that they do not steal issue cycles from the compute warps of their SM
+// sub-partition.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t *bar, uint32_t parity, int *err) {
+    if (mbar_try_wait_hint(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait_hint(bar, parity)) {
+        if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+            if (err) atomicExch(err, ERR_TIMEOUT);
+            return false;
+        }
+        __nanosleep(100);
+    }
+    return true;
+}
+
 // Bounded wait for the phase with the given parity; false (and the error
 // word set) if it did not complete within WAIT_LIMIT_CYCLES.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err) {
@@ -287,6 +316,24 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
         ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// L2 policy for data read once per launch (streamed weights): evict first,
+// so that the stream does not push the kernel's code, the routing tables and
+// the activation records out of L2.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, uint32_t bytes,
+                                              uint64_t *bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
 }
 

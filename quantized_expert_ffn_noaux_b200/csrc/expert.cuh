@@ -590,21 +590,104 @@ struct FastGeo {
     }
 };
 
-template <int BITS>
-__device__ __forceinline__ void gateup_stage_fast(const uint8_t *stage, int RB, const FastGeo &f,
-                                                  int row_base, const LaneAct<BITS, 3> &act,
-                                                  double *part_mat, int ntok) {
-    const int lane = threadIdx.x & 31;
-    double acc[2];
-#pragma unroll
-    for (int k = 0; k < 2; ++k)
-        acc[k] = act.dot(reinterpret_cast<const uint4 *>(stage + (size_t)(f.r0 + k * f.rstep) * RB),
-                         f.vbase);
-    const double tot = warp_sum_rows<2>(acc);
-    if ((lane & 15) == 0) {
-        const int row = f.r0 + (lane >> 4) * f.rstep;
-        part_mat[((row_base + row) * f.slices + f.sl) * ntok] = tot;
+// Ring position: slot and phase parity advance together (no divisions).
+struct RingPos {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void next(int ns) {
+        if (++slot == ns) {
+            slot = 0;
+            phase ^= 1u;
+        }
     }
+};
+
+// The ring as the consumers see it.
+struct RingView {
+    const uint8_t *ring;
+    PipeBars *bars;
+    int ns;
+    int *err;
+    volatile int *abort;
+};
+
+// Consumer side of one whole gate/up item on the fast geometry (SL slices of
+// the row, R = 16 / SL rows a stage, 2 SL stages a matrix): a warp keeps the
+// lane partials of its two rows of every stage in registers and reduces them
+// across the lanes once a matrix, so a stage costs its loads and dots only.
+// False (abort flag set) if a stage wait ran out.
+template <int BITS, int SL>
+__device__ __forceinline__ bool gateup_item_fast(const RingView &rv, RingPos &rp, int RB,
+                                                 const FastGeo &f, const LaneAct<BITS, 3> &act,
+                                                 double *pbuf, size_t part_mat, int ntok) {
+    constexpr int R = 16 / SL, SPM = 32 / R, U = 2 * SPM;
+    constexpr int SHIFT = U == 4 ? 3 : (U == 8 ? 2 : 1);
+    const int lane = threadIdx.x & 31;
+#pragma unroll 1
+    for (int m = 0; m < 2; ++m) {
+        double acc[U];
+#pragma unroll
+        for (int st = 0; st < SPM; ++st) {
+            if (!mbar_wait(&rv.bars->full[rp.slot], rp.phase, rv.err)) {
+                *rv.abort = 1;
+                return false;
+            }
+            const uint8_t *stage = rv.ring + (size_t)rp.slot * PIPE_STAGE_MAX;
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+                acc[2 * st + k] =
+                    act.dot(reinterpret_cast<const uint4 *>(stage + (size_t)(f.r0 + k * f.rstep) * RB), f.vbase);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&rv.bars->empty[rp.slot]);
+            rp.next(rv.ns);
+        }
+        const double tot = warp_sum_rows<U>(acc);
+        if ((lane & ((1 << SHIFT) - 1)) == 0) {
+            const int i = lane >> SHIFT, st = i >> 1, k = i & 1;
+            const int row = st * R + f.r0 + k * f.rstep;
+            pbuf[(size_t)m * part_mat + ((size_t)row * SL + f.sl) * ntok] = tot;
+        }
+    }
+    return true;
+}
+
+// Consumer side of the down rows of one single-token expert when the CTA owns
+// at most 64 output rows: warp w takes rows w + 8 j of the range, whatever
+// stage they arrive in, keeps their lane partials in registers and reduces
+// them once, after the expert's last stage.
+template <int BITS, int VPL>
+__device__ __forceinline__ bool down_expert_fast(const RingView &rv, RingPos &rp, int RB, int VI, int I,
+                                                 int nrows, int subs, int down_rows,
+                                                 const float *scales /* shared, this expert */,
+                                                 const LaneAct<BITS, VPL> &act, int p, float *ebuf,
+                                                 int rows_cap) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    double acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.0;
+    for (int sb = 0; sb < subs; ++sb) {
+        if (!mbar_wait(&rv.bars->full[rp.slot], rp.phase, rv.err)) {
+            *rv.abort = 1;
+            return false;
+        }
+        const int ro = sb * down_rows;
+        const int nr = min(down_rows, nrows - ro);
+        const uint8_t *stage = rv.ring + (size_t)rp.slot * PIPE_STAGE_MAX;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int row = warp + PIPE_CONSUMERS * j;
+            if (row >= ro && row < ro + nr)
+                acc[j] = act.dot(reinterpret_cast<const uint4 *>(stage + (size_t)(row - ro) * RB), 0);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rv.bars->empty[rp.slot]);
+        rp.next(rv.ns);
+    }
+    const double tot = warp_sum_rows<8>(acc);
+    const int row = warp + PIPE_CONSUMERS * (lane >> 2);
+    if ((lane & 3) == 0 && row < nrows)
+        ebuf[(size_t)p * rows_cap + row] = (float)(tot * (double)scales[row]);
+    return true;
 }
 
 // 16-byte asynchronous global -> shared copies (L2 only), completed by
@@ -674,12 +757,11 @@ __device__ __forceinline__ void down_stage(const uint8_t *stage, int RB, int V, 
 // rows).
 template <int BITS, int VPL>
 __device__ __forceinline__ void down_stage_fast(const uint8_t *stage, int RB, int V, int I, int nr,
-                                                const float *scales /* shared */, const uint8_t *rec,
-                                                int p, float *ebuf, int rows_cap, int row_off) {
+                                                const float *scales /* shared */,
+                                                const LaneAct<BITS, VPL> &act, int p, float *ebuf,
+                                                int rows_cap, int row_off) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp >= nr) return;
-    LaneAct<BITS, VPL> act;
-    act.load(rec, I, V, 0);
     for (int g0 = warp; g0 < nr; g0 += 4 * PIPE_CONSUMERS) {
         double acc[4];
 #pragma unroll
@@ -735,7 +817,7 @@ struct DecodeArgs {
 };
 
 struct DecodeSmem {
-    size_t select, idxw, cnt, red, tables, act, ebuf, part, dscale, ring, total;
+    size_t select, idxw, cnt, red, tables, act, ebuf, part, dscale, eptr, ring, total;
 };
 
 __host__ __device__ inline DecodeSmem decode_smem(int T, int H, int I, int E, int S, int G, int k,
@@ -765,21 +847,86 @@ __host__ __device__ inline DecodeSmem decode_smem(int T, int H, int I, int E, in
     d.dscale = o;                         // down-row scales of this CTA, per active expert
     const int amax = (E < T * k ? E : T * k) + S;
     o += align128((size_t)amax * (rows_cap + 4) * 4);
+    d.eptr = o;                           // gate, up, down code pointers per active expert
+    o += align128((size_t)amax * 3 * sizeof(void *));
     d.total = o;
     return d;
 }
 
-// Ring position: slot and phase parity advance together (no divisions).
-struct RingPos {
-    int slot = 0;
-    uint32_t phase = 0;
-    __device__ __forceinline__ void next(int ns) {
-        if (++slot == ns) {
-            slot = 0;
-            phase ^= 1u;
+
+// P4 of the decode kernel: the consumer side of the down stages of this CTA's
+// output rows, one active expert after another.  VPL = vectors per lane of
+// the h activation (1, 2, 4: register-resident activation, loaded once per
+// single-token expert before its first stage wait); VPL = 0 is the generic
+// shared-memory path for any other width.
+struct DownLoop {
+    const int *off;
+    int n_active, subs, ns, down_rows, rows_cap, r0, nrows, RBI, VI, I, rbI;
+    const uint8_t *ring;
+    const float *dscale;
+    const uint8_t *acts;
+    float *ebuf;
+    PipeBars *bars;
+    volatile int *abort;
+    int *err;
+};
+
+template <int BITS, int VPL>
+__device__ __forceinline__ bool down_loop(const DownLoop &d, RingPos &rp) {
+    const int lane = threadIdx.x & 31;
+    const RingView rv{d.ring, d.bars, d.ns, d.err, d.abort};
+    for (int a = 0; a < d.n_active; ++a) {
+        const int p0 = d.off[a], ne = d.off[a + 1] - p0;
+        LaneAct<BITS, (VPL > 0 ? VPL : 1)> act;
+        if constexpr (VPL > 0) {
+            if (ne == 1) act.load(d.acts + (size_t)p0 * d.rbI, d.I, d.VI, 0);
+            if (ne == 1 && d.nrows <= 8 * PIPE_CONSUMERS) {
+                if (!down_expert_fast<BITS, VPL>(rv, rp, d.RBI, d.VI, d.I, d.nrows, d.subs, d.down_rows,
+                                                 d.dscale + a * (d.rows_cap + 4), act, p0, d.ebuf,
+                                                 d.rows_cap))
+                    return false;
+                continue;
+            }
+        }
+        for (int sb = 0; sb < d.subs; ++sb) {
+            if (!mbar_wait(&d.bars->full[rp.slot], rp.phase, d.err)) {
+                *d.abort = 1;
+                return false;
+            }
+            const int rs = d.r0 + sb * d.down_rows;
+            const int nr = min(d.down_rows, d.r0 + d.nrows - rs);
+            const uint8_t *stage = d.ring + (size_t)rp.slot * PIPE_STAGE_MAX;
+            const int ro = rs - d.r0;
+            const float *sc = d.dscale + a * (d.rows_cap + 4) + ro;
+            if constexpr (VPL > 0) {
+                if (ne == 1) {
+                    down_stage_fast<BITS, VPL>(stage, d.RBI, d.VI, d.I, nr, sc, act, p0, d.ebuf, d.rows_cap, ro);
+                } else {
+                    for (int i = 0; i < ne; ++i) {
+                        LaneAct<BITS, VPL> ta;
+                        ta.load(d.acts + (size_t)(p0 + i) * d.rbI, d.I, d.VI, 0);
+                        down_stage_fast<BITS, VPL>(stage, d.RBI, d.VI, d.I, nr, sc, ta, p0 + i, d.ebuf,
+                                                   d.rows_cap, ro);
+                    }
+                }
+            } else {
+                for (int i0 = 0; i0 < ne; i0 += PIPE_PASS_TOK) {
+                    const int nn = min(PIPE_PASS_TOK, ne - i0);
+                    switch (nn) {
+                        case 1: down_stage<BITS, 1>(stage, d.RBI, d.VI, d.I, nr, sc, d.acts, d.rbI, p0 + i0, d.ebuf, d.rows_cap, ro); break;
+                        case 2: down_stage<BITS, 2>(stage, d.RBI, d.VI, d.I, nr, sc, d.acts, d.rbI, p0 + i0, d.ebuf, d.rows_cap, ro); break;
+                        case 3: down_stage<BITS, 3>(stage, d.RBI, d.VI, d.I, nr, sc, d.acts, d.rbI, p0 + i0, d.ebuf, d.rows_cap, ro); break;
+                        default: down_stage<BITS, 4>(stage, d.RBI, d.VI, d.I, nr, sc, d.acts, d.rbI, p0 + i0, d.ebuf, d.rows_cap, ro); break;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&d.bars->empty[rp.slot]);
+            rp.next(d.ns);
         }
     }
-};
+    return true;
+}
 
 // Stage cursor of one CTA: its gate/up items (j-th item, matrix step m), then
 // its down stages (active expert a, row sub-range sb).
@@ -877,18 +1024,24 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         // ------------------------------ producer (lane 0 issues)
         StageCursor cur;
         RingPos rp;
+        const uint64_t pol = l2_evict_first_policy();
         int issued = 0;
         // let the router-weight loads enter the memory queues first
         asm volatile("bar.sync 4, %0;" ::"r"(32 * (PIPE_CONSUMERS + 1)) : "memory");
+        int q_ld = -1;
+        const uint8_t *sh_gate = nullptr, *sh_up = nullptr;
         while (lane == 0 && issued < ns && item_of(cur.j) < n_shared_items) {
             const int item = item_of(cur.j);
             const int q = item / nchunk;
-            const ExpertDev ex = fa.experts[E + q];
-            const QMatDev M = (cur.m < spm) ? ex.gate : ex.up;
+            if (q != q_ld) {
+                sh_gate = fa.experts[E + q].gate.codes;
+                sh_up = fa.experts[E + q].up.codes;
+                q_ld = q;
+            }
             const int row0 = (item - q * nchunk) * 32 + (cur.m % spm) * R;
             mbar_expect_tx(&bars->full[rp.slot], (uint32_t)gu_bytes);
-            bulk_g2s(ring + (size_t)rp.slot * PIPE_STAGE_MAX, M.codes + (size_t)row0 * RB,
-                     (uint32_t)gu_bytes, &bars->full[rp.slot]);
+            bulk_g2s_hint(ring + (size_t)rp.slot * PIPE_STAGE_MAX, (cur.m < spm ? sh_gate : sh_up) + (size_t)row0 * RB,
+                          (uint32_t)gu_bytes, &bars->full[rp.slot], pol);
             ++issued;
             rp.next(ns);
             cur.next(1 << 30, steps, subs);
@@ -898,12 +1051,23 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
                 bulk_prefetch_l2(fa.experts[E + i].down.codes + (size_t)r0 * RBI, (uint32_t)(nrows * RBI));
         __syncwarp();
         named_bar(2, DECODE_THREADS);        // routing tables ready (or aborted)
-        if (lane != 0) return;
         if (*abort) {
-            pipe_drain(bars, ns, issued, 0, fa.err);
+            if (lane == 0) pipe_drain(bars, ns, issued, 0, fa.err);
             return;
         }
         const int n_active = *lw.n_active;
+        // code pointers of every active expert into shared memory, one
+        // parallel round of loads, so that issuing a stage reads no global
+        // memory
+        const uint8_t **ptab = reinterpret_cast<const uint8_t **>(smem + L.eptr);
+        for (int a = lane; a < n_active; a += 32) {
+            const ExpertDev ex = fa.experts[lw.active[a]];
+            ptab[3 * a] = ex.gate.codes;
+            ptab[3 * a + 1] = ex.up.codes;
+            ptab[3 * a + 2] = ex.down.codes;
+        }
+        __syncwarp();
+        if (lane != 0) return;
         const int n_items = n_active * nchunk;
         const int my_items = n_items > (int)blockIdx.x ? (n_items - 1 - (int)blockIdx.x) / G + 1 : 0;
         const int n_total = my_items * steps + n_active * subs;
@@ -916,36 +1080,29 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
             if (!c.down) {
                 int a, e, ch;
                 item_expert_chunk(item_of(c.j), n_active, a, e, ch);
-                if (e < 0) e = lw.active[a];
-                const QMatDev M = (c.m < spm) ? fa.experts[e].gate : fa.experts[e].up;
+                const int up = c.m < spm ? 0 : 1;
                 bytes = (uint32_t)gu_bytes;
-                return M.codes + (size_t)(ch * 32 + (c.m % spm) * R) * RB;
+                return ptab[3 * a + up] + (size_t)(ch * 32 + (c.m - up * spm) * R) * RB;
             }
             const int rs = r0 + c.sb * fa.down_rows;
             const int nr = min(fa.down_rows, r0 + nrows - rs);
             bytes = (uint32_t)(nr * RBI);
-            return fa.experts[lw.active[c.a]].down.codes + (size_t)rs * RBI;
+            return ptab[3 * c.a + 2] + (size_t)rs * RBI;
         };
-        // lookahead cursor for the L2 prefetch, ns stages ahead
-        StageCursor ahead = cur;
-        for (int i = 0; i < ns; ++i) ahead.next(my_items, steps, subs);
+        // No L2 prefetch ahead of the ring: the bulk-copy unit of the SM is
+        // what limits the issue rate, and a prefetch costs it as much as the
+        // copy itself; ns stages in flight already cover the DRAM latency.
         for (int st = issued; st < n_total; ++st) {
-            if (st >= ns && !mbar_wait(&bars->empty[rp.slot], rp.phase ^ 1u, fa.err)) {
+            if (st >= ns && !mbar_wait_sleepy(&bars->empty[rp.slot], rp.phase ^ 1u, fa.err)) {
                 pipe_drain(bars, ns, st, st - ns, fa.err);
                 return;
             }
             uint32_t bytes;
             const uint8_t *src = desc(cur, bytes);
             mbar_expect_tx(&bars->full[rp.slot], bytes);
-            bulk_g2s(ring + (size_t)rp.slot * PIPE_STAGE_MAX, src, bytes, &bars->full[rp.slot]);
-            if (st + ns < n_total) {
-                uint32_t b2;
-                const uint8_t *s2 = desc(ahead, b2);
-                bulk_prefetch_l2(s2, b2);
-            }
+            bulk_g2s_hint(ring + (size_t)rp.slot * PIPE_STAGE_MAX, src, bytes, &bars->full[rp.slot], pol);
             rp.next(ns);
             cur.next(my_items, steps, subs);
-            ahead.next(my_items, steps, subs);
         }
         return;  // the consumers wait for every copy
     }
@@ -969,7 +1126,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
                 const ExpertDev ex = fa.experts[e];
                 const float sg = __ldg(ex.gate.scales + c * 32 + lane);
                 const float su = __ldg(ex.up.scales + c * 32 + lane);
-                if (!mbar_wait(&ebars->part_full[buf], (uint32_t)((n >> 1) & 1), fa.err)) {
+                if (!mbar_wait_sleepy(&ebars->part_full[buf], (uint32_t)((n >> 1) & 1), fa.err)) {
                     ok = false;
                     *abort = 1;
                     break;
@@ -1147,18 +1304,23 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
             break;
         }
         double *pbuf = part + (size_t)buf * 2 * part_mat;
-        for (int ms = 0; ms < steps; ++ms) {
-            if (!mbar_wait(&bars->full[rp.slot], rp.phase, fa.err)) {
-                ok = false;
-                *abort = 1;
-                break;
+        if (fast) {
+            const RingView rv{ring, bars, ns, fa.err, abort};
+            switch (fgeo.slices) {
+                case 1: ok = gateup_item_fast<BITS, 1>(rv, rp, RB, fgeo, act, pbuf, part_mat, ntok); break;
+                case 2: ok = gateup_item_fast<BITS, 2>(rv, rp, RB, fgeo, act, pbuf, part_mat, ntok); break;
+                default: ok = gateup_item_fast<BITS, 4>(rv, rp, RB, fgeo, act, pbuf, part_mat, ntok); break;
             }
-            const uint8_t *stage = ring + (size_t)rp.slot * PIPE_STAGE_MAX;
-            double *pm = pbuf + (ms < spm ? 0 : part_mat);
-            const int row_base = (ms < spm ? ms : ms - spm) * R;
-            if (fast) {
-                gateup_stage_fast<BITS>(stage, RB, fgeo, row_base, act, pm, ntok);
-            } else {
+        } else {
+            for (int ms = 0; ms < steps; ++ms) {
+                if (!mbar_wait(&bars->full[rp.slot], rp.phase, fa.err)) {
+                    ok = false;
+                    *abort = 1;
+                    break;
+                }
+                const uint8_t *stage = ring + (size_t)rp.slot * PIPE_STAGE_MAX;
+                double *pm = pbuf + (ms < spm ? 0 : part_mat);
+                const int row_base = (ms < spm ? ms : ms - spm) * R;
                 for (int i0 = 0; i0 < ne; i0 += PIPE_PASS_TOK) {
                     const int nn = min(PIPE_PASS_TOK, ne - i0);
                     const int *tk = tok + i0;
@@ -1169,10 +1331,10 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
                         default: gateup_stage<BITS, 4>(stage, RB, V, H, geo, row_base, acts, rbH, tk, i0, pm, ntok); break;
                     }
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->empty[rp.slot]);
+                rp.next(ns);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->empty[rp.slot]);
-            rp.next(ns);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&ebars->part_full[buf]);
@@ -1205,41 +1367,13 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
     cp_async_wait_all();
     named_bar(1, 256);
     const int vpl = (VI % 32 == 0) ? VI / 32 : 0;
-    for (int a = 0; a < n_active && ok; ++a) {
-        const int p0 = lw.off[a], ne = lw.off[a + 1] - p0;
-        for (int sb = 0; sb < subs; ++sb) {
-            if (!mbar_wait(&bars->full[rp.slot], rp.phase, fa.err)) {
-                ok = false;
-                *abort = 1;
-                break;
-            }
-            const int rs = r0 + sb * fa.down_rows;
-            const int nr = min(fa.down_rows, r0 + nrows - rs);
-            const uint8_t *stage = ring + (size_t)rp.slot * PIPE_STAGE_MAX;
-            const float *sc = dscale + a * (fa.rows_cap + 4) + (rs - r0);
-            const int ro = rs - r0;
-            if (vpl == 1 || vpl == 2 || vpl == 4) {
-                for (int i = 0; i < ne; ++i) {
-                    const uint8_t *rec = acts + (size_t)(p0 + i) * rbI;
-                    if (vpl == 1) down_stage_fast<BITS, 1>(stage, RBI, VI, I, nr, sc, rec, p0 + i, ebuf, fa.rows_cap, ro);
-                    else if (vpl == 2) down_stage_fast<BITS, 2>(stage, RBI, VI, I, nr, sc, rec, p0 + i, ebuf, fa.rows_cap, ro);
-                    else down_stage_fast<BITS, 4>(stage, RBI, VI, I, nr, sc, rec, p0 + i, ebuf, fa.rows_cap, ro);
-                }
-            } else {
-                for (int i0 = 0; i0 < ne; i0 += PIPE_PASS_TOK) {
-                    const int nn = min(PIPE_PASS_TOK, ne - i0);
-                    switch (nn) {
-                        case 1: down_stage<BITS, 1>(stage, RBI, VI, I, nr, sc, acts, rbI, p0 + i0, ebuf, fa.rows_cap, ro); break;
-                        case 2: down_stage<BITS, 2>(stage, RBI, VI, I, nr, sc, acts, rbI, p0 + i0, ebuf, fa.rows_cap, ro); break;
-                        case 3: down_stage<BITS, 3>(stage, RBI, VI, I, nr, sc, acts, rbI, p0 + i0, ebuf, fa.rows_cap, ro); break;
-                        default: down_stage<BITS, 4>(stage, RBI, VI, I, nr, sc, acts, rbI, p0 + i0, ebuf, fa.rows_cap, ro); break;
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->empty[rp.slot]);
-            rp.next(ns);
-        }
+    DownLoop dl{lw.off, n_active, subs, ns, fa.down_rows, fa.rows_cap, r0, nrows, RBI, VI, I, rbI,
+                ring, dscale, acts, ebuf, bars, abort, fa.err};
+    switch (vpl) {
+        case 1: ok = down_loop<BITS, 1>(dl, rp) && ok; break;
+        case 2: ok = down_loop<BITS, 2>(dl, rp) && ok; break;
+        case 4: ok = down_loop<BITS, 4>(dl, rp) && ok; break;
+        default: ok = down_loop<BITS, 0>(dl, rp) && ok; break;
     }
     named_bar(1, 256);
     if (*abort) return;
