@@ -415,7 +415,8 @@ PipePlan plan_decode(const coli_moe *m, int T) {
     p.pmax = T * (c.top_k + c.n_shared);
     p.rows_cap = (c.hidden + p.grid - 1) / p.grid;
     const int RBI = c.inter * c.wfmt / 8;
-    p.stage_rows = std::max(1, std::min(p.rows_cap, PIPE_STAGE_MAX / RBI));
+    // at most 8 rows per consumer warp in a down stage
+    p.stage_rows = std::max(1, std::min(std::min(p.rows_cap, PIPE_STAGE_MAX / RBI), 8 * PIPE_CONSUMERS));
     const size_t fixed = decode_smem(T, c.hidden, c.inter, c.n_routed, c.n_shared, c.n_group,
                                      c.top_k, p.pmax, g.slices, p.rows_cap, 0).total;
     p.ns = ring_stages(fixed, PIPE_STAGE_MAX);
@@ -485,7 +486,7 @@ template <int BITS>
 coli_status launch_small_path(coli_moe *m, const float *x, int T, float *out, cudaStream_t s) {
     const auto &c = m->cfg;
     const PipePlan p = plan_decode(m, T);
-    auto kern = k_moe_decode<BITS>;
+    auto kern = T == 1 ? k_moe_decode<BITS, 1> : k_moe_decode<BITS, PIPE_MAX_TOK>;
     int occ = 1;
     coli_status st = prepare(m, kern, DECODE_THREADS, p.smem, &occ);
     if (st != COLI_OK) return st;

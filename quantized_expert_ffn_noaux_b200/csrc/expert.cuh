@@ -651,45 +651,6 @@ __device__ __forceinline__ bool gateup_item_fast(const RingView &rv, RingPos &rp
     return true;
 }
 
-// Consumer side of the down rows of one single-token expert when the CTA owns
-// at most 64 output rows: warp w takes rows w + 8 j of the range, whatever
-// stage they arrive in, keeps their lane partials in registers and reduces
-// them once, after the expert's last stage.
-template <int BITS, int VPL>
-__device__ __forceinline__ bool down_expert_fast(const RingView &rv, RingPos &rp, int RB, int VI, int I,
-                                                 int nrows, int subs, int down_rows,
-                                                 const float *scales /* shared, this expert */,
-                                                 const LaneAct<BITS, VPL> &act, int p, float *ebuf,
-                                                 int rows_cap) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    double acc[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = 0.0;
-    for (int sb = 0; sb < subs; ++sb) {
-        if (!mbar_wait(&rv.bars->full[rp.slot], rp.phase, rv.err)) {
-            *rv.abort = 1;
-            return false;
-        }
-        const int ro = sb * down_rows;
-        const int nr = min(down_rows, nrows - ro);
-        const uint8_t *stage = rv.ring + (size_t)rp.slot * PIPE_STAGE_MAX;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int row = warp + PIPE_CONSUMERS * j;
-            if (row >= ro && row < ro + nr)
-                acc[j] = act.dot(reinterpret_cast<const uint4 *>(stage + (size_t)(row - ro) * RB), 0);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&rv.bars->empty[rp.slot]);
-        rp.next(rv.ns);
-    }
-    const double tot = warp_sum_rows<8>(acc);
-    const int row = warp + PIPE_CONSUMERS * (lane >> 2);
-    if ((lane & 3) == 0 && row < nrows)
-        ebuf[(size_t)p * rows_cap + row] = (float)(tot * (double)scales[row]);
-    return true;
-}
-
 // 16-byte asynchronous global -> shared copies (L2 only), completed by
 // cp_async_wait_all.
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
@@ -752,30 +713,87 @@ __device__ __forceinline__ void down_stage(const uint8_t *stage, int RB, int V, 
     }
 }
 
-// Down fast path for one pair: a warp's rows w + 8 k of the stage in groups
-// of four, activation of the pair in registers (VPL vectors per lane, full
-// rows).
-template <int BITS, int VPL>
-__device__ __forceinline__ void down_stage_fast(const uint8_t *stage, int RB, int V, int I, int nr,
+// Down fast path for one pair: warp w takes rows w + 8 i (i < RPW) of the
+// stage, the pair's activation in registers (VPL vectors per lane, full
+// rows), and reduces its RPW lane partials across the lanes at once.  RPW is
+// the stage's rows per warp rounded up, so no dot is issued for a row the
+// stage does not have (except in a shorter last stage).
+template <int BITS, int VPL, int RPW>
+__device__ __forceinline__ void down_stage_fast(const uint8_t *stage, int RB, int nr,
                                                 const float *scales /* shared */,
                                                 const LaneAct<BITS, VPL> &act, int p, float *ebuf,
                                                 int rows_cap, int row_off) {
+    constexpr int U = RPW <= 1 ? 1 : (RPW <= 2 ? 2 : (RPW <= 4 ? 4 : 8));
+    constexpr int SHIFT = U == 1 ? 5 : (U == 2 ? 4 : (U == 4 ? 3 : 2));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (warp >= nr) return;
-    for (int g0 = warp; g0 < nr; g0 += 4 * PIPE_CONSUMERS) {
-        double acc[4];
+    double acc[U];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int row = g0 + PIPE_CONSUMERS * k;
-            acc[k] = (row < nr) ? act.dot(reinterpret_cast<const uint4 *>(stage + (size_t)row * RB), 0)
-                                : 0.0;
+    for (int i = 0; i < U; ++i) {
+        const int row = warp + PIPE_CONSUMERS * i;
+        acc[i] = (i < RPW && row < nr) ? act.dot(reinterpret_cast<const uint4 *>(stage + (size_t)row * RB), 0)
+                                       : 0.0;
+    }
+    const double tot = warp_sum_rows<U>(acc);
+    const int i = lane >> SHIFT;
+    const int row = warp + PIPE_CONSUMERS * i;
+    if ((lane & ((1 << SHIFT) - 1)) == 0 && i < RPW && row < nr)
+        ebuf[(size_t)p * rows_cap + row_off + row] = (float)(tot * (double)scales[row]);
+}
+
+// Down rows of one single-token expert over its SUBS stages (stage sb holds
+// rows sb * down_rows + [0, nr)), warp w taking rows w + 8 i (i < RPW) of
+// each: the lane partials of all SUBS * RPW rows stay in registers and are
+// reduced across the lanes once, after the expert's last stage, instead of
+// once a stage.  Requires down_rows == 8 * RPW (every stage but the last
+// full).  False (abort flag set) if a stage wait ran out.
+template <int BITS, int VPL, int RPW, int SUBS>
+__device__ __forceinline__ bool down_expert_deferred(const RingView &rv, RingPos &rp, int RB, int nrows,
+                                                     const float *scales /* shared, this expert */,
+                                                     const LaneAct<BITS, VPL> &act, int p, float *ebuf,
+                                                     int rows_cap) {
+    constexpr int N = RPW * SUBS;
+    constexpr int U = N <= 4 ? 4 : 8;
+    constexpr int SHIFT = U == 4 ? 3 : 2;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    double acc[U];
+#pragma unroll
+    for (int i = N; i < U; ++i) acc[i] = 0.0;
+#pragma unroll
+    for (int sb = 0; sb < SUBS; ++sb) {
+        if (!mbar_wait(&rv.bars->full[rp.slot], rp.phase, rv.err)) {
+            *rv.abort = 1;
+            return false;
         }
-        const double tot = warp_sum_rows<4>(acc);
-        if ((lane & 7) == 0) {
-            const int row = g0 + PIPE_CONSUMERS * (lane >> 3);
-            if (row < nr)
-                ebuf[(size_t)p * rows_cap + row_off + row] = (float)(tot * (double)scales[row]);
+        const uint8_t *stage = rv.ring + (size_t)rp.slot * PIPE_STAGE_MAX;
+        const int nr = min(8 * RPW, nrows - sb * 8 * RPW);
+#pragma unroll
+        for (int i = 0; i < RPW; ++i) {
+            const int row = warp + PIPE_CONSUMERS * i;
+            acc[sb * RPW + i] =
+                row < nr ? act.dot(reinterpret_cast<const uint4 *>(stage + (size_t)row * RB), 0) : 0.0;
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rv.bars->empty[rp.slot]);
+        rp.next(rv.ns);
+    }
+    const double tot = warp_sum_rows<U>(acc);
+    const int j = lane >> SHIFT, sb = j / RPW, i = j - sb * RPW;
+    const int row = sb * 8 * RPW + warp + PIPE_CONSUMERS * i;
+    if ((lane & ((1 << SHIFT) - 1)) == 0 && j < N && row < nrows)
+        ebuf[(size_t)p * rows_cap + row] = (float)(tot * (double)scales[row]);
+    return true;
+}
+
+template <int BITS, int VPL>
+__device__ __forceinline__ void down_stage_fast_any(int rpw, const uint8_t *stage, int RB, int nr,
+                                                    const float *scales, const LaneAct<BITS, VPL> &act,
+                                                    int p, float *ebuf, int rows_cap, int row_off) {
+    switch (rpw) {
+        case 1: down_stage_fast<BITS, VPL, 1>(stage, RB, nr, scales, act, p, ebuf, rows_cap, row_off); break;
+        case 2: down_stage_fast<BITS, VPL, 2>(stage, RB, nr, scales, act, p, ebuf, rows_cap, row_off); break;
+        case 3: down_stage_fast<BITS, VPL, 3>(stage, RB, nr, scales, act, p, ebuf, rows_cap, row_off); break;
+        case 4: down_stage_fast<BITS, VPL, 4>(stage, RB, nr, scales, act, p, ebuf, rows_cap, row_off); break;
+        default: down_stage_fast<BITS, VPL, 8>(stage, RB, nr, scales, act, p, ebuf, rows_cap, row_off); break;
     }
 }
 
@@ -871,21 +889,32 @@ struct DownLoop {
     int *err;
 };
 
-template <int BITS, int VPL>
+template <int BITS, int VPL, int MAXT>
 __device__ __forceinline__ bool down_loop(const DownLoop &d, RingPos &rp) {
     const int lane = threadIdx.x & 31;
-    const RingView rv{d.ring, d.bars, d.ns, d.err, d.abort};
+    const int rpw = (d.down_rows + PIPE_CONSUMERS - 1) / PIPE_CONSUMERS;
     for (int a = 0; a < d.n_active; ++a) {
         const int p0 = d.off[a], ne = d.off[a + 1] - p0;
         LaneAct<BITS, (VPL > 0 ? VPL : 1)> act;
         if constexpr (VPL > 0) {
-            if (ne == 1) act.load(d.acts + (size_t)p0 * d.rbI, d.I, d.VI, 0);
-            if (ne == 1 && d.nrows <= 8 * PIPE_CONSUMERS) {
-                if (!down_expert_fast<BITS, VPL>(rv, rp, d.RBI, d.VI, d.I, d.nrows, d.subs, d.down_rows,
-                                                 d.dscale + a * (d.rows_cap + 4), act, p0, d.ebuf,
-                                                 d.rows_cap))
-                    return false;
-                continue;
+            if (MAXT == 1 || ne == 1) {
+                act.load(d.acts + (size_t)p0 * d.rbI, d.I, d.VI, 0);
+                // whole expert at once where the stage geometry allows
+                const float *sc_a = d.dscale + a * (d.rows_cap + 4);
+                const RingView rv{d.ring, d.bars, d.ns, d.err, d.abort};
+                int done = -1;
+                if (d.down_rows == 8 * rpw) {
+                    if (rpw == 3 && d.subs == 2)
+                        done = down_expert_deferred<BITS, VPL, 3, 2>(rv, rp, d.RBI, d.nrows, sc_a, act, p0, d.ebuf, d.rows_cap);
+                    else if (rpw == 4 && d.subs == 2)
+                        done = down_expert_deferred<BITS, VPL, 4, 2>(rv, rp, d.RBI, d.nrows, sc_a, act, p0, d.ebuf, d.rows_cap);
+                    else if (rpw == 2 && d.subs <= 4 && d.subs >= 3)
+                        done = d.subs == 3
+                                   ? down_expert_deferred<BITS, VPL, 2, 3>(rv, rp, d.RBI, d.nrows, sc_a, act, p0, d.ebuf, d.rows_cap)
+                                   : down_expert_deferred<BITS, VPL, 2, 4>(rv, rp, d.RBI, d.nrows, sc_a, act, p0, d.ebuf, d.rows_cap);
+                }
+                if (done == 0) return false;
+                if (done == 1) continue;
             }
         }
         for (int sb = 0; sb < d.subs; ++sb) {
@@ -899,16 +928,18 @@ __device__ __forceinline__ bool down_loop(const DownLoop &d, RingPos &rp) {
             const int ro = rs - d.r0;
             const float *sc = d.dscale + a * (d.rows_cap + 4) + ro;
             if constexpr (VPL > 0) {
-                if (ne == 1) {
-                    down_stage_fast<BITS, VPL>(stage, d.RBI, d.VI, d.I, nr, sc, act, p0, d.ebuf, d.rows_cap, ro);
+                if (MAXT == 1 || ne == 1) {
+                    down_stage_fast_any<BITS, VPL>(rpw, stage, d.RBI, nr, sc, act, p0, d.ebuf, d.rows_cap, ro);
                 } else {
                     for (int i = 0; i < ne; ++i) {
                         LaneAct<BITS, VPL> ta;
                         ta.load(d.acts + (size_t)(p0 + i) * d.rbI, d.I, d.VI, 0);
-                        down_stage_fast<BITS, VPL>(stage, d.RBI, d.VI, d.I, nr, sc, ta, p0 + i, d.ebuf,
-                                                   d.rows_cap, ro);
+                        down_stage_fast_any<BITS, VPL>(rpw, stage, d.RBI, nr, sc, ta, p0 + i, d.ebuf,
+                                                       d.rows_cap, ro);
                     }
                 }
+            } else if constexpr (MAXT == 1) {
+                down_stage<BITS, 1>(stage, d.RBI, d.VI, d.I, nr, sc, d.acts, d.rbI, p0, d.ebuf, d.rows_cap, ro);
             } else {
                 for (int i0 = 0; i0 < ne; i0 += PIPE_PASS_TOK) {
                     const int nn = min(PIPE_PASS_TOK, ne - i0);
@@ -955,7 +986,10 @@ struct EpiBars {
     uint64_t part_free[2];   // the epilogue warp finished reading them
 };
 
-template <int BITS>
+// MAXT: the most tokens the instance handles (1, or PIPE_MAX_TOK); the
+// single-token instance carries none of the multi-token code, which keeps the
+// hot loops of every phase compact in the instruction caches.
+template <int BITS, int MAXT>
 __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa) {
     extern __shared__ __align__(128) uint8_t smem[];
     PipeBars *bars = reinterpret_cast<PipeBars *>(smem);
@@ -1174,9 +1208,9 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
     for (int e0 = blockIdx.x; e0 < E; e0 += 2 * G) {
         const int e1 = e0 + G;
         const bool two = e1 < E;
-        double acc[2][PIPE_MAX_TOK];
+        double acc[2][MAXT];
 #pragma unroll
-        for (int t = 0; t < PIPE_MAX_TOK; ++t) acc[0][t] = acc[1][t] = 0.0;
+        for (int t = 0; t < MAXT; ++t) acc[0][t] = acc[1][t] = 0.0;
         const float4 *w40 = reinterpret_cast<const float4 *>(fa.Wr + (int64_t)e0 * H);
         const float4 *w41 = reinterpret_cast<const float4 *>(fa.Wr + (int64_t)(two ? e1 : e0) * H);
         const int H4 = H / 4;
@@ -1190,7 +1224,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
             }
 
 #pragma unroll
-            for (int t = 0; t < PIPE_MAX_TOK; ++t) {
+            for (int t = 0; t < MAXT; ++t) {
                 if (t < T) {
                     float4 xv[4];
 #pragma unroll
@@ -1214,7 +1248,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
             }
         }
 #pragma unroll
-        for (int t = 0; t < PIPE_MAX_TOK; ++t) {
+        for (int t = 0; t < MAXT; ++t) {
             if (t < T) {
                 const double v0 = warp_sum(acc[0][t]);
                 const double v1 = warp_sum(acc[1][t]);
@@ -1295,7 +1329,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         const int p0 = lw.off[a];
         const int ne = min(lw.off[a + 1] - p0, PIPE_MAX_TOK);
         const int *tok = lw.pair_tok + p0;
-        const bool fast = geo.fast && ne == 1;
+        const bool fast = geo.fast && (MAXT == 1 || ne == 1);
         LaneAct<BITS, 3> act;
         if (fast) act.load(acts + (size_t)tok[0] * rbH, H, V, fgeo.vbase);
         if (n >= 2 && !mbar_wait(&ebars->part_free[buf], (uint32_t)(((n >> 1) - 1) & 1), fa.err)) {
@@ -1322,13 +1356,17 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
                 double *pm = pbuf + (ms < spm ? 0 : part_mat);
                 const int row_base = (ms < spm ? ms : ms - spm) * R;
                 for (int i0 = 0; i0 < ne; i0 += PIPE_PASS_TOK) {
-                    const int nn = min(PIPE_PASS_TOK, ne - i0);
+                    const int nn = MAXT == 1 ? 1 : min(PIPE_PASS_TOK, ne - i0);
                     const int *tk = tok + i0;
-                    switch (nn) {
-                        case 1: gateup_stage<BITS, 1>(stage, RB, V, H, geo, row_base, acts, rbH, tk, i0, pm, ntok); break;
-                        case 2: gateup_stage<BITS, 2>(stage, RB, V, H, geo, row_base, acts, rbH, tk, i0, pm, ntok); break;
-                        case 3: gateup_stage<BITS, 3>(stage, RB, V, H, geo, row_base, acts, rbH, tk, i0, pm, ntok); break;
-                        default: gateup_stage<BITS, 4>(stage, RB, V, H, geo, row_base, acts, rbH, tk, i0, pm, ntok); break;
+                    if constexpr (MAXT == 1) {
+                        gateup_stage<BITS, 1>(stage, RB, V, H, geo, row_base, acts, rbH, tk, i0, pm, ntok);
+                    } else {
+                        switch (nn) {
+                            case 1: gateup_stage<BITS, 1>(stage, RB, V, H, geo, row_base, acts, rbH, tk, i0, pm, ntok); break;
+                            case 2: gateup_stage<BITS, 2>(stage, RB, V, H, geo, row_base, acts, rbH, tk, i0, pm, ntok); break;
+                            case 3: gateup_stage<BITS, 3>(stage, RB, V, H, geo, row_base, acts, rbH, tk, i0, pm, ntok); break;
+                            default: gateup_stage<BITS, 4>(stage, RB, V, H, geo, row_base, acts, rbH, tk, i0, pm, ntok); break;
+                        }
                     }
                 }
                 __syncwarp();
@@ -1370,10 +1408,10 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
     DownLoop dl{lw.off, n_active, subs, ns, fa.down_rows, fa.rows_cap, r0, nrows, RBI, VI, I, rbI,
                 ring, dscale, acts, ebuf, bars, abort, fa.err};
     switch (vpl) {
-        case 1: ok = down_loop<BITS, 1>(dl, rp) && ok; break;
-        case 2: ok = down_loop<BITS, 2>(dl, rp) && ok; break;
-        case 4: ok = down_loop<BITS, 4>(dl, rp) && ok; break;
-        default: ok = down_loop<BITS, 0>(dl, rp) && ok; break;
+        case 1: ok = down_loop<BITS, 1, MAXT>(dl, rp) && ok; break;
+        case 2: ok = down_loop<BITS, 2, MAXT>(dl, rp) && ok; break;
+        case 4: ok = down_loop<BITS, 4, MAXT>(dl, rp) && ok; break;
+        default: ok = down_loop<BITS, 0, MAXT>(dl, rp) && ok; break;
     }
     named_bar(1, 256);
     if (*abort) return;
