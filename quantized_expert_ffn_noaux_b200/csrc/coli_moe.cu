@@ -3,6 +3,7 @@
 // Validates arguments, owns the per-handle device workspace, and enqueues the
 // kernels of quant.cuh, route.cuh and expert.cuh on the caller's stream.
 // No call synchronises the host except coli_moe_forward_host.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -18,6 +19,7 @@
 #include "coli_moe.h"
 #include "common.cuh"
 #include "expert.cuh"
+#include "grouped_tc.cuh"
 #include "quant.cuh"
 #include "route.cuh"
 
@@ -94,6 +96,11 @@ struct coli_moe {
     int8_t *hq = nullptr;
     float *hd = nullptr;
     float *e_pairs = nullptr;  // only when max_tokens > SMALL_T
+    bool no_tc = false;        // COLI_NO_TC=1: CUDA-core grouped kernels instead (comparison runs)
+    int8_t *xg = nullptr;      // x codes / scales in pair order (tensor-core path)
+    float *xdg = nullptr;
+    CUtensorMap *maps_dev = nullptr;  // activation maps, then gate/up/down of every expert
+    bool tc_maps = false;
     float *x_in = nullptr, *y_out = nullptr;
     uint8_t *xrec = nullptr, *hrec = nullptr;
     int *err = nullptr;
@@ -119,7 +126,8 @@ struct Layout {
 
 struct WsOffsets {
     size_t s, c, idx, w, bitmap, prefix, counter, n_active, active, off, act_of, pair_tok,
-        pair_slot, tok_pair, xq, xd, hq, hd, e_pairs, x_in, y_out, experts, xrec, hrec, err, gbar;
+        pair_slot, tok_pair, xq, xd, hq, hd, e_pairs, xg, xdg, maps, x_in, y_out, experts, xrec, hrec,
+        err, gbar;
     size_t total;
 };
 
@@ -173,6 +181,11 @@ WsOffsets layout_of(const coli_moe_config &c) {
     o.hq = L.add(P * I);
     o.hd = L.add(P * (I / 32) * 4);
     o.e_pairs = (T > (size_t)SMALL_T) ? L.add(P * H * 4) : 0;
+    // pair-ordered x codes and scales, and the tensor maps, for the grouped
+    // tensor-core path
+    o.xg = (T > (size_t)SMALL_T) ? L.add(P * H) : 0;
+    o.xdg = (T > (size_t)SMALL_T) ? L.add(P * (H / 32) * 4) : 0;
+    o.maps = (T > (size_t)SMALL_T) ? L.add((TC_MAP_W + 3 * (E + S)) * sizeof(CUtensorMap)) : 0;
     o.x_in = L.add(T * H * 4);
     o.y_out = L.add(T * H * 4);
     o.experts = L.add((E + S) * sizeof(ExpertDev));
@@ -544,6 +557,96 @@ coli_status check_handle(coli_moe *m) {
     return COLI_OK;
 }
 
+// 2-D tensor maps through the driver's encoder, fetched from the runtime (no
+// link against the driver library).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    });
+    return fn;
+}
+
+// rows x cols matrix (cols contiguous, row pitch in bytes), box box_rows x box_cols
+bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t rows, uint64_t cols,
+               uint64_t pitch, uint32_t box_rows, uint32_t box_cols) {
+    EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn || !base) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {pitch};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor-core grouped GEMMs for many tokens: both reductions in whole
+// stages of 8 blocks and both row counts in whole tiles.
+bool tc_path_ok(const coli_moe *m) {
+    const auto &c = m->cfg;
+    return m->e_pairs && m->tc_maps && c.hidden % (TC_BPS * 32) == 0 && c.inter % (TC_BPS * 32) == 0 &&
+           c.inter % TC_M == 0 && c.hidden % (2 * TC_M) == 0;
+}
+
+template <int BITS>
+coli_status launch_grouped_tc(coli_moe *m, int T, int down, cudaStream_t s) {
+    const auto &c = m->cfg;
+    const int max_active = std::min(c.n_routed, T * c.top_k) + c.n_shared;
+    const size_t smem = tc_layout(BITS, max_active).total;
+    auto kern = k_grouped_tc<BITS>;
+    int occ = 1;
+    coli_status st = prepare(m, kern, TC_THREADS, smem, &occ);
+    if (st != COLI_OK) return st;
+    if (occ < 1) return fail(COLI_EUNSUPPORTED, "grouped tensor-core kernel does not fit on an SM");
+    TcArgs ta{};
+    ta.ws = m->rw;
+    ta.experts = m->experts_dev;
+    ta.down = down;
+    ta.K = down ? c.inter : c.hidden;
+    ta.I = c.inter;
+    ta.H = c.hidden;
+    ta.maps = m->maps_dev;
+    ta.map_b = down ? TC_MAP_HQ : TC_MAP_XG;
+    ta.map_d = down ? TC_MAP_HD : TC_MAP_XD;
+    ta.hq = m->hq;
+    ta.hd = m->hd;
+    ta.e_pairs = m->e_pairs;
+    ta.err = m->err;
+    Launch L(m, s, down ? "down_tc" : "gateup_tc");
+    kern<<<m->nsm, TC_THREADS, smem, s>>>(ta);
+    return L.done();
+}
+
+template <int BITS>
+coli_status launch_tc_path(coli_moe *m, int T, float *out, cudaStream_t s) {
+    const auto &c = m->cfg;
+    {
+        Launch L(m, s, "gather_pairs");
+        k_gather_pairs<<<m->nsm * 8, 256, 0, s>>>(m->rw, m->xq, m->xd, c.hidden, m->xg, m->xdg);
+        coli_status st = L.done();
+        if (st != COLI_OK) return st;
+    }
+    coli_status st = launch_grouped_tc<BITS>(m, T, 0, s);
+    if (st != COLI_OK) return st;
+    st = launch_grouped_tc<BITS>(m, T, 1, s);
+    if (st != COLI_OK) return st;
+    Launch L(m, s, "combine");
+    const int64_t n = (int64_t)T * c.hidden;
+    int grid = (int)std::min<int64_t>((n + 255) / 256, (int64_t)m->nsm * 8);
+    k_combine<<<grid, 256, 0, s>>>(m->rw, m->e_pairs, T, c.hidden, c.top_k, c.n_shared, out);
+    return L.done();
+}
+
 coli_status forward_impl(coli_moe *m, const float *x, int T, float *out, cudaStream_t s) {
     const auto &c = m->cfg;
     coli_status st;
@@ -560,6 +663,15 @@ coli_status forward_impl(coli_moe *m, const float *x, int T, float *out, cudaStr
     if (st != COLI_OK) return st;
     st = launch_route(m, x, T, m->rw.idx, m->rw.w, 1, s);
     if (st != COLI_OK) return st;
+    if (tc_path_ok(m) && !m->no_tc) {
+        switch (c.wfmt) {
+            case 8: st = launch_tc_path<8>(m, T, out, s); break;
+            case 4: st = launch_tc_path<4>(m, T, out, s); break;
+            default: st = launch_tc_path<2>(m, T, out, s); break;
+        }
+        if (st == COLI_OK) m->last_T = T;
+        return st;
+    }
     const int max_active = std::min(c.n_routed, T * c.top_k) + c.n_shared;
     const int gu_items = max_active * (c.inter / ROWS_PER_ITEM);
     switch (c.wfmt) {
@@ -734,6 +846,7 @@ coli_status coli_moe_create(const coli_moe_config *cfg, const float *router_w, c
     m->bias = bias;
     cudaGetDevice(&m->device);
     m->nsm = sm_count();
+    m->no_tc = getenv("COLI_NO_TC") && strcmp(getenv("COLI_NO_TC"), "1") == 0;
     const WsOffsets o = layout_of(*cfg);
     if (getenv("COLI_FAULT") && strcmp(getenv("COLI_FAULT"), "alloc") == 0) {
         delete m;
@@ -766,6 +879,9 @@ coli_status coli_moe_create(const coli_moe_config *cfg, const float *router_w, c
     m->hq = (int8_t *)(b + o.hq);
     m->hd = (float *)(b + o.hd);
     m->e_pairs = o.e_pairs ? (float *)(b + o.e_pairs) : nullptr;
+    m->xg = o.xg ? (int8_t *)(b + o.xg) : nullptr;
+    m->xdg = o.xdg ? (float *)(b + o.xdg) : nullptr;
+    m->maps_dev = o.maps ? (CUtensorMap *)(b + o.maps) : nullptr;
     m->x_in = (float *)(b + o.x_in);
     m->y_out = (float *)(b + o.y_out);
     m->experts_dev = (ExpertDev *)(b + o.experts);
@@ -776,6 +892,32 @@ coli_status coli_moe_create(const coli_moe_config *cfg, const float *router_w, c
     e = cudaMemset(m->ws_base, 0, o.total);
     if (e == cudaSuccess)
         e = cudaMemcpy(m->experts_dev, host.data(), sizeof(ExpertDev) * n, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && m->maps_dev) {
+        // the tensor-core path's maps; any shape or alignment the copy engine
+        // refuses leaves that path off (the CUDA-core grouped kernels run)
+        const uint64_t H = cfg->hidden, I = cfg->inter, P = (uint64_t)cfg->max_tokens * (cfg->top_k + cfg->n_shared);
+        const int bits = cfg->wfmt;
+        std::vector<CUtensorMap> maps(TC_MAP_W + 3 * n);
+        bool ok = H % (TC_BPS * 32) == 0 && I % (TC_BPS * 32) == 0;
+        const uint32_t rawrow = (uint32_t)(TC_BPS * 32 * bits / 8);
+        ok = ok && encode_2d(&maps[TC_MAP_XG], CU_TENSOR_MAP_DATA_TYPE_UINT8, m->xg, P, H, H, TC_N, TC_BPS * 32);
+        ok = ok && encode_2d(&maps[TC_MAP_XD], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, m->xdg, P, H / 32, H / 8, TC_N, TC_BPS);
+        ok = ok && encode_2d(&maps[TC_MAP_HQ], CU_TENSOR_MAP_DATA_TYPE_UINT8, m->hq, P, I, I, TC_N, TC_BPS * 32);
+        ok = ok && encode_2d(&maps[TC_MAP_HD], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, m->hd, P, I / 32, I / 8, TC_N, TC_BPS);
+        for (int i = 0; ok && i < n; ++i) {
+            const uint64_t gu_pitch = H * bits / 8, dn_pitch = I * bits / 8;
+            ok = encode_2d(&maps[TC_MAP_W + 3 * i], CU_TENSOR_MAP_DATA_TYPE_UINT8, host[i].gate.codes, I, gu_pitch,
+                           gu_pitch, TC_M, rawrow) &&
+                 encode_2d(&maps[TC_MAP_W + 3 * i + 1], CU_TENSOR_MAP_DATA_TYPE_UINT8, host[i].up.codes, I,
+                           gu_pitch, gu_pitch, TC_M, rawrow) &&
+                 encode_2d(&maps[TC_MAP_W + 3 * i + 2], CU_TENSOR_MAP_DATA_TYPE_UINT8, host[i].down.codes, H,
+                           dn_pitch, dn_pitch, TC_M, rawrow);
+        }
+        if (ok) {
+            e = cudaMemcpy(m->maps_dev, maps.data(), sizeof(CUtensorMap) * maps.size(), cudaMemcpyHostToDevice);
+            m->tc_maps = e == cudaSuccess;
+        }
+    }
     if (e != cudaSuccess) {
         cudaFree(m->ws_base);
         delete m;
