@@ -100,6 +100,7 @@ struct coli_moe {
     int8_t *xg = nullptr;      // x codes / scales in pair order (tensor-core path)
     float *xdg = nullptr;
     CUtensorMap *maps_dev = nullptr;  // activation maps, then gate/up/down of every expert
+    double *corr_x = nullptr, *corr_h = nullptr;  // per-pair weight-offset shares
     bool tc_maps = false;
     float *x_in = nullptr, *y_out = nullptr;
     uint8_t *xrec = nullptr, *hrec = nullptr;
@@ -126,7 +127,8 @@ struct Layout {
 
 struct WsOffsets {
     size_t s, c, idx, w, bitmap, prefix, counter, n_active, active, off, act_of, pair_tok,
-        pair_slot, tok_pair, xq, xd, hq, hd, e_pairs, xg, xdg, maps, x_in, y_out, experts, xrec, hrec,
+        pair_slot, tok_pair, xq, xd, hq, hd, e_pairs, xg, xdg, maps, corr_x, corr_h, x_in, y_out, experts,
+        xrec, hrec,
         err, gbar;
     size_t total;
 };
@@ -186,6 +188,8 @@ WsOffsets layout_of(const coli_moe_config &c) {
     o.xg = (T > (size_t)SMALL_T) ? L.add(P * H) : 0;
     o.xdg = (T > (size_t)SMALL_T) ? L.add(P * (H / 32) * 4) : 0;
     o.maps = (T > (size_t)SMALL_T) ? L.add((TC_MAP_W + 3 * (E + S)) * sizeof(CUtensorMap)) : 0;
+    o.corr_x = (T > (size_t)SMALL_T) ? L.add(P * 8) : 0;
+    o.corr_h = (T > (size_t)SMALL_T) ? L.add(P * 8) : 0;
     o.x_in = L.add(T * H * 4);
     o.y_out = L.add(T * H * 4);
     o.experts = L.add((E + S) * sizeof(ExpertDev));
@@ -618,6 +622,7 @@ coli_status launch_grouped_tc(coli_moe *m, int T, int down, cudaStream_t s) {
     ta.maps = m->maps_dev;
     ta.map_b = down ? TC_MAP_HQ : TC_MAP_XG;
     ta.map_d = down ? TC_MAP_HD : TC_MAP_XD;
+    ta.corr = down ? m->corr_h : m->corr_x;
     ta.hq = m->hq;
     ta.hd = m->hd;
     ta.e_pairs = m->e_pairs;
@@ -630,14 +635,27 @@ coli_status launch_grouped_tc(coli_moe *m, int T, int down, cudaStream_t s) {
 template <int BITS>
 coli_status launch_tc_path(coli_moe *m, int T, float *out, cudaStream_t s) {
     const auto &c = m->cfg;
+    const double off = BITS == 4 ? 8.0 : 2.0;  // unsigned weight operands: code + off
     {
         Launch L(m, s, "gather_pairs");
         k_gather_pairs<<<m->nsm * 8, 256, 0, s>>>(m->rw, m->xq, m->xd, c.hidden, m->xg, m->xdg);
         coli_status st = L.done();
         if (st != COLI_OK) return st;
     }
+    if (BITS != 8) {
+        Launch L(m, s, "pair_offsets");
+        k_pair_offsets<<<m->nsm * 8, 256, 0, s>>>(m->rw, m->xg, m->xdg, c.hidden, off, m->corr_x);
+        coli_status st = L.done();
+        if (st != COLI_OK) return st;
+    }
     coli_status st = launch_grouped_tc<BITS>(m, T, 0, s);
     if (st != COLI_OK) return st;
+    if (BITS != 8) {
+        Launch L(m, s, "pair_offsets");
+        k_pair_offsets<<<m->nsm * 8, 256, 0, s>>>(m->rw, m->hq, m->hd, c.inter, off, m->corr_h);
+        st = L.done();
+        if (st != COLI_OK) return st;
+    }
     st = launch_grouped_tc<BITS>(m, T, 1, s);
     if (st != COLI_OK) return st;
     Launch L(m, s, "combine");
@@ -882,6 +900,8 @@ coli_status coli_moe_create(const coli_moe_config *cfg, const float *router_w, c
     m->xg = o.xg ? (int8_t *)(b + o.xg) : nullptr;
     m->xdg = o.xdg ? (float *)(b + o.xdg) : nullptr;
     m->maps_dev = o.maps ? (CUtensorMap *)(b + o.maps) : nullptr;
+    m->corr_x = o.corr_x ? (double *)(b + o.corr_x) : nullptr;
+    m->corr_h = o.corr_h ? (double *)(b + o.corr_h) : nullptr;
     m->x_in = (float *)(b + o.x_in);
     m->y_out = (float *)(b + o.y_out);
     m->experts_dev = (ExpertDev *)(b + o.experts);
@@ -899,19 +919,19 @@ coli_status coli_moe_create(const coli_moe_config *cfg, const float *router_w, c
         const int bits = cfg->wfmt;
         std::vector<CUtensorMap> maps(TC_MAP_W + 3 * n);
         bool ok = H % (TC_BPS * 32) == 0 && I % (TC_BPS * 32) == 0;
-        const uint32_t rawrow = (uint32_t)(TC_BPS * 32 * bits / 8);
-        ok = ok && encode_2d(&maps[TC_MAP_XG], CU_TENSOR_MAP_DATA_TYPE_UINT8, m->xg, P, H, H, TC_N, TC_BPS * 32);
+        const uint32_t gb = (uint32_t)tc_group_bytes(bits);
+        ok = ok && encode_2d(&maps[TC_MAP_XG], CU_TENSOR_MAP_DATA_TYPE_UINT8, m->xg, P, H, H, TC_N, 32);
         ok = ok && encode_2d(&maps[TC_MAP_XD], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, m->xdg, P, H / 32, H / 8, TC_N, TC_BPS);
-        ok = ok && encode_2d(&maps[TC_MAP_HQ], CU_TENSOR_MAP_DATA_TYPE_UINT8, m->hq, P, I, I, TC_N, TC_BPS * 32);
+        ok = ok && encode_2d(&maps[TC_MAP_HQ], CU_TENSOR_MAP_DATA_TYPE_UINT8, m->hq, P, I, I, TC_N, 32);
         ok = ok && encode_2d(&maps[TC_MAP_HD], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, m->hd, P, I / 32, I / 8, TC_N, TC_BPS);
         for (int i = 0; ok && i < n; ++i) {
             const uint64_t gu_pitch = H * bits / 8, dn_pitch = I * bits / 8;
             ok = encode_2d(&maps[TC_MAP_W + 3 * i], CU_TENSOR_MAP_DATA_TYPE_UINT8, host[i].gate.codes, I, gu_pitch,
-                           gu_pitch, TC_M, rawrow) &&
+                           gu_pitch, TC_M, gb) &&
                  encode_2d(&maps[TC_MAP_W + 3 * i + 1], CU_TENSOR_MAP_DATA_TYPE_UINT8, host[i].up.codes, I,
-                           gu_pitch, gu_pitch, TC_M, rawrow) &&
+                           gu_pitch, gu_pitch, TC_M, gb) &&
                  encode_2d(&maps[TC_MAP_W + 3 * i + 2], CU_TENSOR_MAP_DATA_TYPE_UINT8, host[i].down.codes, H,
-                           dn_pitch, dn_pitch, TC_M, rawrow);
+                           dn_pitch, dn_pitch, TC_M, gb);
         }
         if (ok) {
             e = cudaMemcpy(m->maps_dev, maps.data(), sizeof(CUtensorMap) * maps.size(), cudaMemcpyHostToDevice);

@@ -11,16 +11,17 @@
 // value = (float)(acc * row_scale).
 //
 // One CTA per SM, persistent over items (active expert, row tile, 32-token
-// tile), 12 warps:
+// tile), 24 warps:
 //   warp 0      producer: four 2-D TMA copies a stage of 8 blocks -- the two
 //               128-row tiles of raw weight codes (int8/int4/int2), and the 32
 //               pair rows of activation codes and of block scales (pair order:
 //               x is gathered by pair first, h is written that way)
-//   warps 1-2   expand one block at a time into the K-major canonical layout
-//               (signed int8), scales to fp64
-//   warp 3      TMEM owner; one thread issues the two MMAs of a block
-//   warps 4-11  epilogue: warp 4+q reads TMEM lane quarter q of A tile 0,
-//               warp 8+q of A tile 1; fp64 promotion; the item's end
+//   warp 1      TMEM owner; one thread issues the two MMAs of a block
+//   warps 2, 3, 20-23   expand one block at a time into the K-major
+//               canonical layout, scales to fp64
+//   warps 4-19  epilogue: warp 4 + q + 4 m + 8 h reads TMEM lane quarter q
+//               of A tile m, token columns 16 h .. 16 h + 15; exact fp64
+//               promotion (the fp64 pipe bounds the kernel); the item's end
 // Gate/up items pair the gate and up rows of a 128-row tile and end in
 // SwiGLU + Q8_0(h); down items pair two 128-row tiles of the down matrix and
 // end in the per-pair outputs e[p][row].  Every wait is bounded.
@@ -39,9 +40,16 @@ constexpr int TC_BPS = 8;        // 32-blocks per stage
 constexpr int TC_STAGES = 2;     // raw stages
 constexpr int TC_SLOTS = 4;      // canonical operand slots (one block each)
 constexpr int TC_BUFS = 4;       // TMEM accumulator buffers (64 columns each)
-constexpr int TC_THREADS = 384;
+constexpr int TC_THREADS = 768;
+constexpr int TC_EXPAND_WARPS = 6;  // warps 2, 3 and 20-23
+constexpr int TC_EPI_WARPS = 16;    // warps 4-19
+constexpr int TC_EXPAND_THREADS = 32 * TC_EXPAND_WARPS;
 constexpr int TC_TMEM_COLS = 256;
 constexpr int TC_OP_BYTES = 2 * TC_M * 32 + TC_N * 32;  // A0, A1, B of one block
+// Raw weight codes land block-major: column groups of tc_group_bytes(BITS)
+// bytes (one 32-block, two for int2) of all 128 rows, so that the expanding
+// lanes read consecutive rows (no bank conflicts).
+__host__ __device__ constexpr int tc_group_bytes(int bits) { return 4 * bits < 16 ? 16 : 4 * bits; }
 
 struct TcBars {
     uint64_t raw_full[TC_STAGES], raw_empty[TC_STAGES];
@@ -97,6 +105,7 @@ struct TcArgs {
     int I;                  // intermediate size (h layout)
     int H;                  // hidden size (e_pairs layout)
     int map_b, map_d;       // maps of the activation codes and scales [pairs][K], [pairs][K/32]
+    const double *corr;     // per pair: the weight offset's share (int4 / int2), see k_pair_offsets
     int8_t *hq;             // gate/up outputs
     float *hd;
     float *e_pairs;         // down output [pairs][H]
@@ -111,15 +120,21 @@ __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr) {
     return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(128 >> 4) << 16) |
            ((uint64_t)(256 >> 4) << 32) | (1ull << 46);
 }
-// kind::i8, signed A and B, s32 accumulator, K-major A and B, M = 128, N = TC_N
-constexpr uint32_t TC_IDESC = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TC_N >> 3) << 17) |
-                              ((uint32_t)(TC_M >> 4) << 24);
+// kind::i8, s32 accumulator, K-major A and B, M = 128, N = TC_N; B (the
+// activation codes) signed, A signed for int8 weights and unsigned for int4 /
+// int2 (codes stored as code + 8 / code + 2, see tc_expand)
+template <int BITS>
+__host__ __device__ constexpr uint32_t tc_idesc() {
+    return (2u << 4) | ((BITS == 8 ? 1u : 0u) << 7) | (1u << 10) | ((uint32_t)(TC_N >> 3) << 17) |
+           ((uint32_t)(TC_M >> 4) << 24);
+}
 
+template <int BITS>
 __device__ __forceinline__ void tc_mma(uint32_t dtmem, uint64_t da, uint64_t db) {
     asm volatile(
         "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
         " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(dtmem),
-        "l"(da), "l"(db), "r"(TC_IDESC), "r"(0u));
+        "l"(da), "l"(db), "r"(tc_idesc<BITS>()), "r"(0u));
 }
 __device__ __forceinline__ void tc_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -136,6 +151,14 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&v)[32]) {
           "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
           "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
           "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -168,6 +191,41 @@ __global__ void k_gather_pairs(RouteWs ws, const int8_t *__restrict__ xq, const 
     }
 }
 
+// Per pair, the unsigned-weight offset's share of every row's sum:
+// off * sum_b (sum of the pair's codes in block b) * d_b, in fp64, blocks in
+// order (deterministic).  One CTA per pair; codes [pairs][K] in pair order.
+__global__ void k_pair_offsets(RouteWs ws, const int8_t *__restrict__ q, const float *__restrict__ d, int K,
+                               double off, double *__restrict__ out) {
+    __shared__ double part[256];
+    const int np = ws.off[*ws.n_active];
+    const int nb = K / COLI_QBLK;
+    for (int p = blockIdx.x; p < np; p += gridDim.x) {
+        double acc = 0.0;
+        for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+            const int4 *c = reinterpret_cast<const int4 *>(q + (size_t)p * K + (size_t)b * COLI_QBLK);
+            const int4 c0 = c[0], c1 = c[1];
+            int sx = 0;
+            sx = __dp4a(c0.x, 0x01010101, sx);
+            sx = __dp4a(c0.y, 0x01010101, sx);
+            sx = __dp4a(c0.z, 0x01010101, sx);
+            sx = __dp4a(c0.w, 0x01010101, sx);
+            sx = __dp4a(c1.x, 0x01010101, sx);
+            sx = __dp4a(c1.y, 0x01010101, sx);
+            sx = __dp4a(c1.z, 0x01010101, sx);
+            sx = __dp4a(c1.w, 0x01010101, sx);
+            acc = fma((double)sx, (double)d[(size_t)p * nb + b], acc);
+        }
+        part[threadIdx.x] = acc;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double t = 0.0;
+            for (int i = 0; i < (int)blockDim.x; ++i) t += part[i];
+            out[p] = off * t;
+        }
+        __syncthreads();
+    }
+}
+
 // Bounded wait that also gives up once another role has aborted.
 __device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, TcBars *tb, int *err) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -183,9 +241,12 @@ __device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, TcBars *
     }
 }
 
-// One weight row's 32-wide block, raw codes -> 32 signed int8 (two 16-byte
-// halves of the canonical layout).  Element k of a row: int8 byte k; int4
-// nibble k (low nibble first); int2 crumb k (low bits first).
+// One weight row's 32-wide block, raw codes -> 32 MMA operand bytes (two
+// 16-byte halves of the canonical layout).  Element k of a row: int8 byte k
+// (signed, as is); int4 nibble k (low nibble first) as the unsigned code + 8;
+// int2 crumb k (low bits first) as the unsigned code + 2.  The offset's
+// contribution, off * sum_k x_k per block, is removed per pair at the end
+// (tc_pair_offsets).
 template <int BITS>
 __device__ __forceinline__ void tc_expand(const uint8_t *raw, uint4 &c0, uint4 &c1) {
     if constexpr (BITS == 8) {
@@ -197,9 +258,9 @@ __device__ __forceinline__ void tc_expand(const uint8_t *raw, uint4 &c0, uint4 &
         uint32_t o[8];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            // nibble v -> (v ^ 8) + 0x78, top bit flipped: the signed value
-            const uint32_t lo = ((((ws[i] & 0x0F0F0F0Fu) ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u);
-            const uint32_t hi = (((((ws[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u);
+            // nibble v (two's complement) -> v ^ 8 = code + 8
+            const uint32_t lo = (ws[i] & 0x0F0F0F0Fu) ^ 0x08080808u;
+            const uint32_t hi = ((ws[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
             o[2 * i] = prmt(lo, hi, 0x5140);      // elements 8i+0..3
             o[2 * i + 1] = prmt(lo, hi, 0x7362);  // elements 8i+4..7
         }
@@ -214,7 +275,7 @@ __device__ __forceinline__ void tc_expand(const uint8_t *raw, uint4 &c0, uint4 &
             uint32_t c[4];
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                c[s] = ((((ws[i] >> (2 * s)) & 0x03030303u) ^ 0x02020202u) + 0x7E7E7E7Eu) ^ 0x80808080u;
+                c[s] = ((ws[i] >> (2 * s)) & 0x03030303u) ^ 0x02020202u;  // code + 2
             const uint32_t t01l = prmt(c[0], c[1], 0x5140), t23l = prmt(c[2], c[3], 0x5140);
             const uint32_t t01h = prmt(c[0], c[1], 0x7362), t23h = prmt(c[2], c[3], 0x7362);
             o[4 * i + 0] = prmt(t01l, t23l, 0x5410);
@@ -248,17 +309,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
     if (tid == 0) {
         for (int i = 0; i < TC_STAGES; ++i) {
             mbar_init(&tb->raw_full[i], 1);
-            mbar_init(&tb->raw_empty[i], 2);
+            mbar_init(&tb->raw_empty[i], TC_EXPAND_WARPS);
         }
         for (int i = 0; i < TC_SLOTS; ++i) {
-            mbar_init(&tb->op_full[i], 2);
+            mbar_init(&tb->op_full[i], TC_EXPAND_WARPS);
             mbar_init(&tb->op_empty[i], 1);
         }
         for (int i = 0; i < TC_BUFS; ++i) {
             mbar_init(&tb->tm_full[i], 1);
-            mbar_init(&tb->tm_empty[i], 8);
-            mbar_init(&tb->dd_full[i], 2);
-            mbar_init(&tb->dd_empty[i], 8);
+            mbar_init(&tb->tm_empty[i], TC_EPI_WARPS);
+            mbar_init(&tb->dd_full[i], TC_EXPAND_WARPS);
+            mbar_init(&tb->dd_empty[i], TC_EPI_WARPS);
         }
         tb->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -284,7 +345,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
             tb->n_items = run;
         }
     }
-    if (warp == 3) {
+    if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(&tb->taddr)),
                      "r"(TC_TMEM_COLS));
@@ -351,9 +412,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
                     uint64_t *bar = &tb->raw_full[slot];
                     mbar_expect_tx(bar, (uint32_t)(L.rawA + L.rawB + L.rawD));
                     const int k0 = s * TC_BPS * 32;  // first element of the stage
-                    tma2d(raw, a.maps + mp[0], k0 * BITS / 8, r0[0], bar);
-                    tma2d(raw + (size_t)TC_M * rawrow, a.maps + mp[1], k0 * BITS / 8, r0[1], bar);
-                    tma2d(raw + L.rawA, a.maps + a.map_b, k0, p0, bar);
+                    constexpr int GB = tc_group_bytes(BITS);
+#pragma unroll
+                    for (int m = 0; m < 2; ++m)
+                        for (int g = 0; g < rawrow / GB; ++g)
+                            tma2d(raw + (size_t)m * TC_M * rawrow + (size_t)g * TC_M * GB, a.maps + mp[m],
+                                  k0 * BITS / 8 + g * GB, r0[m], bar);
+                    for (int j = 0; j < TC_BPS; ++j)
+                        tma2d(raw + L.rawA + j * (TC_N * 32), a.maps + a.map_b, k0 + 32 * j, p0, bar);
                     tma2d(raw + L.rawA + L.rawB, a.maps + a.map_d, k0 / COLI_QBLK, p0, bar);
                 }
             }
@@ -365,9 +431,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
             }
         }
         __syncwarp();
-    } else if (warp == 1 || warp == 2) {
+    } else if (warp == 2 || warp == 3 || warp >= 4 + TC_EPI_WARPS) {
         // ------------------------------------------------------------ expand
-        const int et = tid - 32;  // 0..63
+        const int et = warp < 4 ? tid - 64 : tid - 32 * (4 + TC_EPI_WARPS) + 64;  // 0..191
         int sc = 0, blk = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -389,18 +455,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
                     }
                     uint8_t *op = smem + L.op + (size_t)cs * TC_OP_BYTES;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int i = et + 64 * q;  // 0..255: A tile i / 128, row i % 128
+                    for (int q = 0; q < 2; ++q) {
+                        const int i = et + TC_EXPAND_THREADS * q;  // 0..255: A tile i / 128, row i % 128
+                        if (i >= 2 * TC_M) break;
                         const int m = i >> 7, r = i & 127;
                         uint4 c0, c1;
-                        tc_expand<BITS>(raw + (size_t)i * rawrow + j * (32 * BITS / 8), c0, c1);
+                        constexpr int GB = tc_group_bytes(BITS), BPG = GB / (4 * BITS);
+                        tc_expand<BITS>(raw + (size_t)m * TC_M * rawrow + (size_t)(j / BPG) * TC_M * GB +
+                                            (size_t)r * GB + (j % BPG) * (4 * BITS),
+                                        c0, c1);
                         uint8_t *dst = op + m * (TC_M * 32);
                         *reinterpret_cast<uint4 *>(dst + tc_canon(r, 0)) = c0;
                         *reinterpret_cast<uint4 *>(dst + tc_canon(r, 1)) = c1;
                     }
-                    {
+                    if (et < 2 * TC_N) {
                         const int t = et >> 1, hf = et & 1;
-                        const uint4 v = *reinterpret_cast<const uint4 *>(rawB + (size_t)t * TC_BPS * 32 + j * 32 + hf * 16);
+                        const uint4 v = *reinterpret_cast<const uint4 *>(rawB + j * (TC_N * 32) + t * 32 + hf * 16);
                         *reinterpret_cast<uint4 *>(op + 2 * TC_M * 32 + tc_canon(t, hf)) = v;
                     }
                     if (et < TC_N) {
@@ -418,7 +488,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
                 if (lane == 0) mbar_arrive(&tb->raw_empty[slot]);
             }
         }
-    } else if (warp == 3) {
+    } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
         int blk = 0;
         bool ok = true;
@@ -434,8 +504,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
                     tc_fence_after();
                     const uint32_t op = smem_u32(smem + L.op + (size_t)cs * TC_OP_BYTES);
                     const uint64_t dB = tc_desc(op + 2 * TC_M * 32);
-                    tc_mma(tmem + (uint32_t)(bf * 64), tc_desc(op), dB);
-                    tc_mma(tmem + (uint32_t)(bf * 64 + 32), tc_desc(op + TC_M * 32), dB);
+                    tc_mma<BITS>(tmem + (uint32_t)(bf * 64), tc_desc(op), dB);
+                    tc_mma<BITS>(tmem + (uint32_t)(bf * 64 + 32), tc_desc(op + TC_M * 32), dB);
                     tc_commit(&tb->op_empty[cs]);
                     tc_commit(&tb->tm_full[bf]);
                 }
@@ -449,7 +519,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
-        const int e = warp - 4, m = e >> 2, q = warp & 3;
+        constexpr int NH = TC_N / 2;  // token columns of one warp
+        const int e = warp - 4, m = (e >> 2) & 1, hh = e >> 3, q = warp & 3;
+        const int c0 = hh * NH;       // first token column
         int blk = 0;
         bool ok = true;
         float *xch = reinterpret_cast<float *>(smem + L.xch) + (size_t)q * TC_N * 32;
@@ -458,9 +530,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
             decode_item(item, ae, rt, tt);
             const int p0 = a.ws.off[ae] + tt * TC_N;
             const int nt = min(TC_N, a.ws.off[ae + 1] - p0);
-            double acc[TC_N];
+            double acc[NH];
 #pragma unroll
-            for (int t = 0; t < TC_N; ++t) acc[t] = 0.0;
+            for (int t = 0; t < NH; ++t) acc[t] = 0.0;
             for (int k = 0; k < nblk; ++k, ++blk) {
                 const int bf = blk % TC_BUFS;
                 const uint32_t ph = (uint32_t)(blk / TC_BUFS) & 1u;
@@ -469,8 +541,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
                     break;
                 }
                 tc_fence_after();
-                uint32_t v[32];
-                tc_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(bf * 64 + m * 32), v);
+                uint32_t v[NH];
+                tc_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(bf * 64 + m * 32 + c0), v);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tb->tm_empty[bf]);
@@ -478,9 +550,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
                     ok = false;
                     break;
                 }
-                const double2 *dd = reinterpret_cast<const double2 *>(smem + L.dd) + bf * (TC_N / 2);
+                const double2 *dd = reinterpret_cast<const double2 *>(smem + L.dd) + bf * (TC_N / 2) + c0 / 2;
 #pragma unroll
-                for (int t = 0; t < TC_N; t += 2) {
+                for (int t = 0; t < NH; t += 2) {
                     const double2 d2 = dd[t >> 1];
                     acc[t] = fma((double)(int)v[t], d2.x, acc[t]);
                     acc[t + 1] = fma((double)(int)v[t + 1], d2.y, acc[t + 1]);
@@ -493,28 +565,32 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
             a_rows(ae, rt, m, scales, row0, map_unused);
             const int r = row0 + 32 * q + lane;
             const double sw = (double)__ldg(scales + r);
+            if (BITS != 8) {
+#pragma unroll
+                for (int t = 0; t < NH; ++t) acc[t] -= (c0 + t < nt) ? __ldg(a.corr + p0 + c0 + t) : 0.0;
+            }
             if (a.down) {
                 if (!ok) break;
 #pragma unroll
-                for (int t = 0; t < TC_N; ++t)
-                    if (t < nt) a.e_pairs[(size_t)(p0 + t) * a.H + r] = (float)(acc[t] * sw);
+                for (int t = 0; t < NH; ++t)
+                    if (c0 + t < nt) a.e_pairs[(size_t)(p0 + c0 + t) * a.H + r] = (float)(acc[t] * sw);
             } else {
-                // u through shared memory to the gate warp of the same quarter;
-                // both warps of the pair pass both barriers even after an
-                // abort, so that neither waits for the other forever
-                if (m == 1 && ok) {
+                // g and u of this quarter through shared memory (each warp its
+                // 16 columns); the gate warp of a half then finishes those
+                // columns.  Both warps of a pair pass both barriers even after
+                // an abort, so that neither waits for the other forever.
+                float *xg = xch + 4 * TC_N * 32;
+                if (ok) {
+                    float *dst = m ? xch : xg;
 #pragma unroll
-                    for (int t = 0; t < TC_N; ++t) xch[t * 32 + lane] = (float)(acc[t] * sw);
+                    for (int t = 0; t < NH; ++t) dst[(c0 + t) * 32 + lane] = (float)(acc[t] * sw);
                 }
-                asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
+                const int bar_id = 1 + q + 4 * hh;
+                asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
                 if (m == 0 && ok && !*(volatile int *)&tb->abort) {
-                    // g beside u (static indices keep acc in registers)
-                    float *xg = xch + 4 * TC_N * 32;
-#pragma unroll
-                    for (int t = 0; t < TC_N; ++t) xg[t * 32 + lane] = (float)(acc[t] * sw);
-                    __syncwarp();
                     const int nb = a.I / COLI_QBLK;
-                    for (int t = 0; t < nt; ++t) {
+                    const int tend = min(c0 + NH, nt);
+                    for (int t = c0; t < tend; ++t) {
                         const float g = xg[t * 32 + lane];
                         const float u = xch[t * 32 + lane];
                         const double gd = (double)g;
@@ -526,14 +602,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
                         if (lane == 0) a.hd[(size_t)p * nb + (r >> 5)] = dh;
                     }
                 }
-                asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
+                asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
                 if (!ok) break;
             }
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 3) {
+    if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_TMEM_COLS));
     }
