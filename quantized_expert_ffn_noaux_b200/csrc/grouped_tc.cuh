@@ -39,11 +39,12 @@ constexpr int TC_N = 32;         // tokens per item
 constexpr int TC_BPS = 8;        // 32-blocks per stage
 constexpr int TC_STAGES = 2;     // raw stages
 constexpr int TC_SLOTS = 4;      // canonical operand slots (one block each)
-constexpr int TC_BUFS = 4;       // TMEM accumulator buffers (64 columns each)
+constexpr int TC_BUFS = 4;       // TMEM accumulator buffers (64 columns each) and scale slots
 constexpr int TC_THREADS = 768;
 constexpr int TC_EXPAND_WARPS = 6;  // warps 2, 3 and 20-23
 constexpr int TC_EPI_WARPS = 16;    // warps 4-19
 constexpr int TC_EXPAND_THREADS = 32 * TC_EXPAND_WARPS;
+constexpr int TC_EXPAND_GROUP = TC_EXPAND_THREADS / 2;  // two groups take alternate blocks
 constexpr int TC_TMEM_COLS = 256;
 constexpr int TC_OP_BYTES = 2 * TC_M * 32 + TC_N * 32;  // A0, A1, B of one block
 // Raw weight codes land block-major: column groups of tc_group_bytes(BITS)
@@ -312,13 +313,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
             mbar_init(&tb->raw_empty[i], TC_EXPAND_WARPS);
         }
         for (int i = 0; i < TC_SLOTS; ++i) {
-            mbar_init(&tb->op_full[i], TC_EXPAND_WARPS);
+            mbar_init(&tb->op_full[i], TC_EXPAND_WARPS / 2);
             mbar_init(&tb->op_empty[i], 1);
         }
         for (int i = 0; i < TC_BUFS; ++i) {
             mbar_init(&tb->tm_full[i], 1);
             mbar_init(&tb->tm_empty[i], TC_EPI_WARPS);
-            mbar_init(&tb->dd_full[i], TC_EXPAND_WARPS);
+            mbar_init(&tb->dd_full[i], TC_EXPAND_WARPS / 2);
             mbar_init(&tb->dd_empty[i], TC_EPI_WARPS);
         }
         tb->abort = 0;
@@ -434,6 +435,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
     } else if (warp == 2 || warp == 3 || warp >= 4 + TC_EPI_WARPS) {
         // ------------------------------------------------------------ expand
         const int et = warp < 4 ? tid - 64 : tid - 32 * (4 + TC_EPI_WARPS) + 64;  // 0..191
+        const int grp = et / TC_EXPAND_GROUP, gt = et % TC_EXPAND_GROUP;        // whole warps per group
         int sc = 0, blk = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -447,6 +449,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
                 const uint8_t *rawB = raw + L.rawA;
                 const float *rawD = reinterpret_cast<const float *>(raw + L.rawA + L.rawB);
                 for (int j = 0; j < TC_BPS && ok; ++j, ++blk) {
+                    if ((blk & 1) != grp) continue;
                     const int cs = blk % TC_SLOTS, db = blk % TC_BUFS;
                     if (!tc_wait(&tb->op_empty[cs], ((uint32_t)(blk / TC_SLOTS) & 1u) ^ 1u, tb, a.err) ||
                         !tc_wait(&tb->dd_empty[db], ((uint32_t)(blk / TC_BUFS) & 1u) ^ 1u, tb, a.err)) {
@@ -455,8 +458,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
                     }
                     uint8_t *op = smem + L.op + (size_t)cs * TC_OP_BYTES;
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const int i = et + TC_EXPAND_THREADS * q;  // 0..255: A tile i / 128, row i % 128
+                    for (int q = 0; q < (2 * TC_M + TC_EXPAND_GROUP - 1) / TC_EXPAND_GROUP; ++q) {
+                        const int i = gt + TC_EXPAND_GROUP * q;  // 0..255: A tile i / 128, row i % 128
                         if (i >= 2 * TC_M) break;
                         const int m = i >> 7, r = i & 127;
                         uint4 c0, c1;
@@ -468,14 +471,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
                         *reinterpret_cast<uint4 *>(dst + tc_canon(r, 0)) = c0;
                         *reinterpret_cast<uint4 *>(dst + tc_canon(r, 1)) = c1;
                     }
-                    if (et < 2 * TC_N) {
-                        const int t = et >> 1, hf = et & 1;
+                    if (gt < 2 * TC_N) {
+                        const int t = gt >> 1, hf = gt & 1;
                         const uint4 v = *reinterpret_cast<const uint4 *>(rawB + j * (TC_N * 32) + t * 32 + hf * 16);
                         *reinterpret_cast<uint4 *>(op + 2 * TC_M * 32 + tc_canon(t, hf)) = v;
                     }
-                    if (et < TC_N) {
+                    if (gt < TC_N) {
                         double *dd = reinterpret_cast<double *>(smem + L.dd) + db * TC_N;
-                        dd[et] = (double)rawD[et * TC_BPS + j];
+                        dd[gt] = (double)rawD[gt * TC_BPS + j];
                     }
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
