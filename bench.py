@@ -68,6 +68,14 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def sm_max_mhz():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["sm_max_mhz"])
+    except Exception:
+        return 1965.0
+
+
 def source_sha():
     h = hashlib.sha256()
     d = os.path.join(ROOT, "quantized_expert_ffn_noaux_b200", "csrc")
@@ -290,7 +298,28 @@ def run_coli(args, cfg, rank, world, device):
         alg = None
     peak, peak_kind = peaks()
     roofline = None
-    if alg is not None:
+    if dom.startswith("gateup_tc") or dom.startswith("down_tc"):
+        # The tensor-core grouped GEMMs are bound by the exact promotion of
+        # every 32-block product (int -> fp64 convert + fp64 FMA), not by
+        # HBM: that fp64 work against the fp64 lanes of the part.
+        H, I = cfg["hidden"], cfg["inter"]
+        pairs = T * (cfg["top_k"] + cfg["n_shared"])
+        if dom.startswith("gateup"):
+            blocks, macs = pairs * 2 * I * (H // 32), pairs * 2 * I * H
+        else:
+            blocks, macs = pairs * H * (I // 32), pairs * H * I
+        nsm = torch.cuda.get_device_properties(device).multi_processor_count
+        sm_mhz = sm_max_mhz()
+        peak_fp64 = nsm * 64 * sm_mhz * 1e6 / 1e9
+        ach = 2 * blocks / (avg_ms / 1e3) / 1e9
+        roofline = {"bound": "alu", "achieved": round(ach, 1), "peak": round(peak_fp64, 1), "unit": "Gop/s",
+                    "frac": round(ach / peak_fp64, 4), "traffic": recorded_traffic(dom, cfg["name"]),
+                    "kernel": dom, "ops": "fp64 promotion of 32-block int8 products: convert + FMA",
+                    "peak_source": "derived: %d SMs x 64 fp64 lanes x %.0f MHz (max SM clock)" % (nsm, sm_mhz),
+                    "ops_per_launch": int(2 * blocks), "avg_launch_ms": round(avg_ms, 5),
+                    "int8_tensor_tops": round(2 * macs / (avg_ms / 1e3) / 1e12, 2),
+                    "int8_tensor_frac_of_nominal_4500": round(2 * macs / (avg_ms / 1e3) / 1e12 / 4500.0, 4)}
+    elif alg is not None:
         ach = alg / (avg_ms / 1e3) / 1e9
         roofline = {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
                     "frac": round(ach / peak, 4), "traffic": recorded_traffic(dom, cfg["name"]),
