@@ -1214,10 +1214,13 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         const float4 *w40 = reinterpret_cast<const float4 *>(fa.Wr + (int64_t)e0 * H);
         const float4 *w41 = reinterpret_cast<const float4 *>(fa.Wr + (int64_t)(two ? e1 : e0) * H);
         const int H4 = H / 4;
-        for (int i0 = tid; i0 < H4; i0 += 4 * 256) {
-            float4 wa[4], wb[4];
+        // all of a thread's router-weight loads in flight at once where the
+        // registers allow (hidden 6144: 6 float4 per thread and expert)
+        constexpr int LU = MAXT == 1 ? 6 : 4;
+        for (int i0 = tid; i0 < H4; i0 += LU * 256) {
+            float4 wa[LU], wb[LU];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < LU; ++u) {
                 const int i = i0 + u * 256;
                 wa[u] = (i < H4) ? __ldg(w40 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
                 wb[u] = (i < H4) ? __ldg(w41 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1226,15 +1229,15 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
 #pragma unroll
             for (int t = 0; t < MAXT; ++t) {
                 if (t < T) {
-                    float4 xv[4];
+                    float4 xv[LU];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < LU; ++u) {
                         const int i = i0 + u * 256;
                         xv[u] = (i < H4) ? __ldg(reinterpret_cast<const float4 *>(fa.x + (int64_t)t * H) + i)
                                          : make_float4(0.f, 0.f, 0.f, 0.f);
                     }
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < LU; ++u) {
                         acc[0][t] = fma((double)xv[u].x, (double)wa[u].x, acc[0][t]);
                         acc[0][t] = fma((double)xv[u].y, (double)wa[u].y, acc[0][t]);
                         acc[0][t] = fma((double)xv[u].z, (double)wa[u].z, acc[0][t]);

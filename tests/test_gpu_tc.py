@@ -64,3 +64,16 @@ def test_grouped_tensor_core_repeat_is_bit_identical():
     assert (a == b).all()
     assert gl.handle.device_status() == 0
     gl.close()
+
+
+def test_cuda_core_grouped_path_on_tensor_core_shapes(monkeypatch):
+    """COLI_NO_TC=1 (read when the handle is created) keeps the CUDA-core
+    grouped kernels on shapes the tensor-core path would take: both many-token
+    paths meet the same bar on the same inputs."""
+    monkeypatch.setenv("COLI_NO_TC", "1")
+    cfg = _cfg(bits=4, seed=47)
+    gl = GpuLayer(cfg, max_tokens=40)
+    x = synth.tokens(cfg, T=40, device=DEV)
+    assert not _ran_tensor_cores(gl, x)
+    compare_forward(gl, x)
+    gl.close()
