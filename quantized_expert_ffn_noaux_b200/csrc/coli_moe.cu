@@ -105,7 +105,8 @@ struct coli_moe {
     float *x_in = nullptr, *y_out = nullptr;
     uint8_t *xrec = nullptr, *hrec = nullptr;
     int *err = nullptr;
-    unsigned long long *gbar = nullptr;  // grid-barrier arrival counter of the decode kernel
+    unsigned long long *gbar = nullptr;
+    int *hcnt = nullptr;  // per active expert: gate/up items done (decode kernel)  // grid-barrier arrival counter of the decode kernel
     int last_T = 0;
     std::map<const void *, int> occ_cache;  // kernel -> CTAs per SM (attributes already set)
     // profiling
@@ -129,7 +130,7 @@ struct WsOffsets {
     size_t s, c, idx, w, bitmap, prefix, counter, n_active, active, off, act_of, pair_tok,
         pair_slot, tok_pair, xq, xd, hq, hd, e_pairs, xg, xdg, maps, corr_x, corr_h, x_in, y_out, experts,
         xrec, hrec,
-        err, gbar;
+        err, gbar, hcnt;
     size_t total;
 };
 
@@ -197,6 +198,7 @@ WsOffsets layout_of(const coli_moe_config &c) {
     o.hrec = L.add(P * (size_t)rec_bytes((int)I));
     o.err = L.add(4);
     o.gbar = L.add(8);
+    o.hcnt = L.add((E + S) * 4);
     o.total = L.total;
     return o;
 }
@@ -532,6 +534,7 @@ coli_status launch_small_path(coli_moe *m, const float *x, int T, float *out, cu
     fa.out = out;
     fa.err = m->err;
     fa.gbar = m->gbar;
+    fa.hcnt = m->hcnt;
     fa.ns = p.ns;
     fa.pmax = p.pmax;
     fa.rows_cap = p.rows_cap;
@@ -909,6 +912,7 @@ coli_status coli_moe_create(const coli_moe_config *cfg, const float *router_w, c
     m->hrec = (uint8_t *)(b + o.hrec);
     m->err = (int *)(b + o.err);
     m->gbar = (unsigned long long *)(b + o.gbar);
+    m->hcnt = (int *)(b + o.hcnt);
     e = cudaMemset(m->ws_base, 0, o.total);
     if (e == cudaSuccess)
         e = cudaMemcpy(m->experts_dev, host.data(), sizeof(ExpertDev) * n, cudaMemcpyHostToDevice);

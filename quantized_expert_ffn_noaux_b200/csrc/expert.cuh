@@ -412,7 +412,7 @@ struct PipeBars {
     int abort;
 };
 
-__host__ __device__ inline size_t pipe_hdr_bytes() { return (sizeof(PipeBars) + 8 + 32 + 127) & ~(size_t)127; }
+__host__ __device__ inline size_t pipe_hdr_bytes() { return (sizeof(PipeBars) + 8 + 64 + 127) & ~(size_t)127; }
 __host__ __device__ inline size_t align128(size_t x) { return (x + 127) & ~(size_t)127; }
 
 // Gate/up rows per stage: a power of two dividing 32 with R * rowbytes <= 24 KB.
@@ -694,12 +694,13 @@ __device__ inline bool grid_barrier(unsigned long long *count, unsigned nblocks,
 // starting at pair p; writes e = (float)(sum * row scale) to ebuf.
 template <int BITS, int NT>
 __device__ __forceinline__ void down_stage(const uint8_t *stage, int RB, int V, int I, int nr,
-                                           const float *scales, const uint8_t *hacts, int rbI,
+                                           const float *scales, const uint8_t *recs, int rbI,
                                            int p, float *ebuf, int rows_cap, int row_off) {
+    // records of the NT tokens at recs + i rbI; their outputs at pairs p + i
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint8_t *rec[NT];
 #pragma unroll
-    for (int i = 0; i < NT; ++i) rec[i] = hacts + (size_t)(p + i) * rbI;
+    for (int i = 0; i < NT; ++i) rec[i] = recs + (size_t)i * rbI;
     for (int row = warp; row < nr; row += PIPE_CONSUMERS) {
         const float sc = scales[row];
         double acc[NT];
@@ -803,15 +804,17 @@ __device__ __forceinline__ void down_stage_fast_any(int rpw, const uint8_t *stag
 // kernel: the shared experts' gate/up rows (issued while routing is still in
 // progress: they need none), the routed experts' gate/up rows, then the down
 // rows of this CTA's output-row range for every active expert (they need no
-// h, so they stream across the second grid barrier).
+// h, so they stream while the gate/up items finish elsewhere).
 //   P1  fp64 logits of experts b, b + grid, ...; Q8_0(x) records of a share
-//       of the blocks, to global memory.            -- grid barrier 1 --
+//       of the blocks, to global memory.            -- grid barrier --
 //   P2  every CTA copies the records, selects every token's experts and
 //       builds the batch-union tables in shared memory (CTA 0 publishes them).
-//   P3  gate/up items + SwiGLU + Q8_0(h) records, to global memory.
-//                                                   -- grid barrier 2 --
-//   P4  h records of every pair into shared memory; down rows of every active
-//       expert; fp64 combine of this CTA's rows, shared experts first.
+//   P3  gate/up items + SwiGLU + Q8_0(h) records, to global memory; each item
+//       adds one to its expert's count.
+//   P4  experts in the down order (shared first): once an expert's count is
+//       complete, the epilogue warp copies its h records into one of two
+//       shared slots and the consumers run its down rows; then the fp64
+//       combine of this CTA's rows, shared experts first.
 struct DecodeArgs {
     const float *x;
     const float *Wr;
@@ -829,6 +832,7 @@ struct DecodeArgs {
     float *out;
     int *err;
     unsigned long long *gbar;   // grid-barrier arrival counter
+    int *hcnt;                  // per active expert: gate/up items whose h records are written
     int ns, pmax;
     int rows_cap;       // output rows per CTA (max) in P4
     int down_rows;      // down rows per stage
@@ -855,7 +859,7 @@ __host__ __device__ inline DecodeSmem decode_smem(int T, int H, int I, int E, in
     d.tables = o;
     o += align128((size_t)(3 * (E + S) + 1 + 3 * pmax + 4) * 4);
     d.act = o;
-    const size_t xa = (size_t)T * rec_bytes(H), ha = (size_t)pmax * rec_bytes(I);
+    const size_t xa = (size_t)T * rec_bytes(H), ha = (size_t)2 * T * rec_bytes(I);
     o += align128(xa > ha ? xa : ha);
     d.ebuf = o;
     o += align128((size_t)pmax * rows_cap * 4);
@@ -877,32 +881,55 @@ __host__ __device__ inline DecodeSmem decode_smem(int T, int H, int I, int E, in
 // the h activation (1, 2, 4: register-resident activation, loaded once per
 // single-token expert before its first stage wait); VPL = 0 is the generic
 // shared-memory path for any other width.
+struct EpiBars {
+    uint64_t part_full[2];   // the 8 consumer warps finished an item's partials
+    uint64_t part_free[2];   // the epilogue warp finished reading them
+    uint64_t h_full[2];      // an expert's h records are in its shared slot
+    uint64_t h_empty[2];     // the 8 consumer warps are done with that slot
+};
+
 struct DownLoop {
     const int *off;
-    int n_active, subs, ns, down_rows, rows_cap, r0, nrows, RBI, VI, I, rbI;
+    int n_active, S, T, subs, ns, down_rows, rows_cap, r0, nrows, RBI, VI, I, rbI;
     const uint8_t *ring;
     const float *dscale;
-    const uint8_t *acts;
+    const uint8_t *acts;     // two slots of T h records each, filled by the epilogue warp
     float *ebuf;
     PipeBars *bars;
+    EpiBars *ebars;
     volatile int *abort;
     int *err;
 };
+
+// Order of the down phase: the shared experts first (their h is complete
+// earliest: their gate/up items come first), then the routed ones.
+__device__ __forceinline__ int down_slot(int q, int n_active, int S) {
+    return q < S ? n_active - S + q : q - S;
+}
 
 template <int BITS, int VPL, int MAXT>
 __device__ __forceinline__ bool down_loop(const DownLoop &d, RingPos &rp) {
     const int lane = threadIdx.x & 31;
     const int rpw = (d.down_rows + PIPE_CONSUMERS - 1) / PIPE_CONSUMERS;
-    for (int a = 0; a < d.n_active; ++a) {
+    for (int q = 0; q < d.n_active; ++q) {
+        const int a = down_slot(q, d.n_active, d.S);
         const int p0 = d.off[a], ne = d.off[a + 1] - p0;
+        // this expert's h records: slot q & 1, filled once all its gate/up
+        // items (any CTA's) are written
+        const uint8_t *recs = d.acts + (size_t)(q & 1) * d.T * d.rbI;
+        if (!mbar_wait(&d.ebars->h_full[q & 1], (uint32_t)(q >> 1) & 1u, d.err)) {
+            *d.abort = 1;
+            return false;
+        }
+        bool expert_ok = true;
         LaneAct<BITS, (VPL > 0 ? VPL : 1)> act;
+        int done = -1;
         if constexpr (VPL > 0) {
             if (MAXT == 1 || ne == 1) {
-                act.load(d.acts + (size_t)p0 * d.rbI, d.I, d.VI, 0);
+                act.load(recs, d.I, d.VI, 0);
                 // whole expert at once where the stage geometry allows
                 const float *sc_a = d.dscale + a * (d.rows_cap + 4);
                 const RingView rv{d.ring, d.bars, d.ns, d.err, d.abort};
-                int done = -1;
                 if (d.down_rows == 8 * rpw) {
                     if (rpw == 3 && d.subs == 2)
                         done = down_expert_deferred<BITS, VPL, 3, 2>(rv, rp, d.RBI, d.nrows, sc_a, act, p0, d.ebuf, d.rows_cap);
@@ -914,13 +941,13 @@ __device__ __forceinline__ bool down_loop(const DownLoop &d, RingPos &rp) {
                                    : down_expert_deferred<BITS, VPL, 2, 4>(rv, rp, d.RBI, d.nrows, sc_a, act, p0, d.ebuf, d.rows_cap);
                 }
                 if (done == 0) return false;
-                if (done == 1) continue;
             }
         }
-        for (int sb = 0; sb < d.subs; ++sb) {
+        for (int sb = 0; done != 1 && sb < d.subs; ++sb) {
             if (!mbar_wait(&d.bars->full[rp.slot], rp.phase, d.err)) {
                 *d.abort = 1;
-                return false;
+                expert_ok = false;
+                break;
             }
             const int rs = d.r0 + sb * d.down_rows;
             const int nr = min(d.down_rows, d.r0 + d.nrows - rs);
@@ -933,21 +960,22 @@ __device__ __forceinline__ bool down_loop(const DownLoop &d, RingPos &rp) {
                 } else {
                     for (int i = 0; i < ne; ++i) {
                         LaneAct<BITS, VPL> ta;
-                        ta.load(d.acts + (size_t)(p0 + i) * d.rbI, d.I, d.VI, 0);
+                        ta.load(recs + (size_t)i * d.rbI, d.I, d.VI, 0);
                         down_stage_fast_any<BITS, VPL>(rpw, stage, d.RBI, nr, sc, ta, p0 + i, d.ebuf,
                                                        d.rows_cap, ro);
                     }
                 }
             } else if constexpr (MAXT == 1) {
-                down_stage<BITS, 1>(stage, d.RBI, d.VI, d.I, nr, sc, d.acts, d.rbI, p0, d.ebuf, d.rows_cap, ro);
+                down_stage<BITS, 1>(stage, d.RBI, d.VI, d.I, nr, sc, recs, d.rbI, p0, d.ebuf, d.rows_cap, ro);
             } else {
                 for (int i0 = 0; i0 < ne; i0 += PIPE_PASS_TOK) {
                     const int nn = min(PIPE_PASS_TOK, ne - i0);
+                    const uint8_t *r = recs + (size_t)i0 * d.rbI;
                     switch (nn) {
-                        case 1: down_stage<BITS, 1>(stage, d.RBI, d.VI, d.I, nr, sc, d.acts, d.rbI, p0 + i0, d.ebuf, d.rows_cap, ro); break;
-                        case 2: down_stage<BITS, 2>(stage, d.RBI, d.VI, d.I, nr, sc, d.acts, d.rbI, p0 + i0, d.ebuf, d.rows_cap, ro); break;
-                        case 3: down_stage<BITS, 3>(stage, d.RBI, d.VI, d.I, nr, sc, d.acts, d.rbI, p0 + i0, d.ebuf, d.rows_cap, ro); break;
-                        default: down_stage<BITS, 4>(stage, d.RBI, d.VI, d.I, nr, sc, d.acts, d.rbI, p0 + i0, d.ebuf, d.rows_cap, ro); break;
+                        case 1: down_stage<BITS, 1>(stage, d.RBI, d.VI, d.I, nr, sc, r, d.rbI, p0 + i0, d.ebuf, d.rows_cap, ro); break;
+                        case 2: down_stage<BITS, 2>(stage, d.RBI, d.VI, d.I, nr, sc, r, d.rbI, p0 + i0, d.ebuf, d.rows_cap, ro); break;
+                        case 3: down_stage<BITS, 3>(stage, d.RBI, d.VI, d.I, nr, sc, r, d.rbI, p0 + i0, d.ebuf, d.rows_cap, ro); break;
+                        default: down_stage<BITS, 4>(stage, d.RBI, d.VI, d.I, nr, sc, r, d.rbI, p0 + i0, d.ebuf, d.rows_cap, ro); break;
                     }
                 }
             }
@@ -955,6 +983,10 @@ __device__ __forceinline__ bool down_loop(const DownLoop &d, RingPos &rp) {
             if (lane == 0) mbar_arrive(&d.bars->empty[rp.slot]);
             rp.next(d.ns);
         }
+        if (!expert_ok) return false;
+        // the slot may be refilled
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&d.ebars->h_empty[q & 1]);
     }
     return true;
 }
@@ -979,11 +1011,6 @@ struct StageCursor {
             ++a;
         }
     }
-};
-
-struct EpiBars {
-    uint64_t part_full[2];   // the 8 consumer warps finished an item's partials
-    uint64_t part_free[2];   // the epilogue warp finished reading them
 };
 
 // MAXT: the most tokens the instance handles (1, or PIPE_MAX_TOK); the
@@ -1033,6 +1060,8 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&ebars->part_full[i], PIPE_CONSUMERS);
             mbar_init(&ebars->part_free[i], 1);
+            mbar_init(&ebars->h_full[i], 1);
+            mbar_init(&ebars->h_empty[i], PIPE_CONSUMERS);
         }
     }
     pipe_init(bars, ns);
@@ -1121,7 +1150,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
             const int rs = r0 + c.sb * fa.down_rows;
             const int nr = min(fa.down_rows, r0 + nrows - rs);
             bytes = (uint32_t)(nr * RBI);
-            return ptab[3 * c.a + 2] + (size_t)rs * RBI;
+            return ptab[3 * down_slot(c.a, n_active, S) + 2] + (size_t)rs * RBI;
         };
         // No L2 prefetch ahead of the ring: the bulk-copy unit of the SM is
         // what limits the issue rate, and a prefetch costs it as much as the
@@ -1181,12 +1210,54 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
                                              fa.hq + (int64_t)pr * I, fa.hd + (int64_t)pr * (I / COLI_QBLK));
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&ebars->part_free[buf]);
+                if (lane == 0) {
+                    mbar_arrive(&ebars->part_free[buf]);
+                    __threadfence();  // the item's h records before its count
+                    atomicAdd(fa.hcnt + a, 1);
+                }
             }
         }
-        // let the consumers enter grid barrier 2 once every h record is written
-        __syncwarp();
-        asm volatile("bar.arrive 3, %0;" ::"r"(32 * (PIPE_CONSUMERS + 1)) : "memory");
+        // then the h records of every active expert, in the down order, into
+        // two shared slots, each once all its gate/up items (any CTA's) are
+        // counted -- this replaces a grid barrier: a CTA starts its down rows
+        // of an expert as soon as that expert's h is complete
+        if (ok && !*abort) {
+            const int n_active = *lw.n_active;
+            for (int q = 0; q < n_active; ++q) {
+                const int a = down_slot(q, n_active, S), slot = q & 1;
+                if (q >= 2 && !mbar_wait_sleepy(&ebars->h_empty[slot], (uint32_t)(((q >> 1) - 1) & 1), fa.err)) {
+                    *abort = 1;
+                    break;
+                }
+                int ready = 1;
+                if (lane == 0) {
+                    const long long t0 = clock64();
+                    while ((int)ld_acquire_u32(reinterpret_cast<const unsigned *>(fa.hcnt + a)) < nchunk) {
+                        if (*abort) {
+                            ready = 0;
+                            break;
+                        }
+                        if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+                            atomicExch(fa.err, ERR_TIMEOUT);
+                            ready = 0;
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                }
+                ready = __shfl_sync(0xffffffffu, ready, 0);
+                if (!ready) {
+                    *abort = 1;
+                    break;
+                }
+                const int p0 = lw.off[a], ne = lw.off[a + 1] - p0;
+                const uint4 *src = reinterpret_cast<const uint4 *>(fa.hrec + (size_t)p0 * rbI);
+                uint4 *dst = reinterpret_cast<uint4 *>(acts + (size_t)slot * T * rbI);
+                for (int i = lane; i < ne * rbI / 16; i += 32) dst[i] = __ldcg(src + i);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ebars->h_full[slot]);
+            }
+        }
         return;
     }
 
@@ -1273,6 +1344,8 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         }
         named_bar(1, 256);
     }
+    if (blockIdx.x == 0)  // this launch's h-record counts start at zero
+        for (int i = tid; i < (E < T * k ? E : T * k) + S; i += 256) fa.hcnt[i] = 0;
     for (int blk = blockIdx.x * PIPE_CONSUMERS + warp; blk < T * nbH; blk += G * PIPE_CONSUMERS) {
         const int t = blk / nbH, b = blk % nbH;
         const float v = __ldg(fa.x + (int64_t)t * H + b * COLI_QBLK + lane);
@@ -1311,11 +1384,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         }
     }
     named_bar(2, DECODE_THREADS);        // tables ready: release producer and epilogue warp
-    if (*abort) {
-        __syncwarp();
-        asm volatile("bar.sync 3, %0;" ::"r"(32 * (PIPE_CONSUMERS + 1)) : "memory");
-        return;
-    }
+    if (*abort) return;
 
     // P3: gate/up items; partials go to the epilogue warp through part_full /
     // part_free (two buffers)
@@ -1381,7 +1450,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         if (lane == 0) mbar_arrive(&ebars->part_full[buf]);
     }
     // down-row scales of this CTA's rows for every active expert (they need
-    // no h): 4-byte async copies, waited for with the h records below
+    // no h): 4-byte async copies
     if (!*abort) {
         const int ds = fa.rows_cap + 4;
         for (int i = tid; i < n_active * nrows; i += 256) {
@@ -1392,24 +1461,13 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
                          : "memory");
         }
     }
-    // grid barrier 2: every h record is written (the epilogue warp arrives on
-    // barrier 3 when its last record is out; the producer keeps streaming)
-    __syncwarp();
-    asm volatile("bar.sync 3, %0;" ::"r"(32 * (PIPE_CONSUMERS + 1)) : "memory");
-    if (tid == 0) flags[0] = (!*abort && grid_barrier(fa.gbar, G, fa.err)) ? 1 : 0;
-    named_bar(1, 256);
-    if (!flags[0]) {
-        *abort = 1;
-        return;
-    }
-    // P4: h records of every pair, down rows, combine
-    const int n_pairs = lw.off[n_active];
-    for (int i = tid; i < n_pairs * rbI / 16; i += 256) cp_async16(acts + 16 * i, fa.hrec + 16 * i);
     cp_async_wait_all();
     named_bar(1, 256);
+    if (*abort) return;
+    // P4: down rows of every active expert as its h arrives, then the combine
     const int vpl = (VI % 32 == 0) ? VI / 32 : 0;
-    DownLoop dl{lw.off, n_active, subs, ns, fa.down_rows, fa.rows_cap, r0, nrows, RBI, VI, I, rbI,
-                ring, dscale, acts, ebuf, bars, abort, fa.err};
+    DownLoop dl{lw.off, n_active, S, T, subs, ns, fa.down_rows, fa.rows_cap, r0, nrows, RBI, VI, I, rbI,
+                ring, dscale, acts, ebuf, bars, ebars, abort, fa.err};
     switch (vpl) {
         case 1: ok = down_loop<BITS, 1, MAXT>(dl, rp) && ok; break;
         case 2: ok = down_loop<BITS, 2, MAXT>(dl, rp) && ok; break;
