@@ -141,7 +141,14 @@ coli_status coli_router(coli_moe *m, const float *x, int T, int32_t *idx, float 
  *   out[t] = sum_shared e_s(x_t) + sum_j w[t][j] * e_{idx[t][j]}(x_t)
  *   e(x) = down . Q8_0( SwiGLU( gate . Q8_0(x), up . Q8_0(x) ) )
  * x [T][H] fp32 (device), out [T][H] fp32 (device, overwritten; must not
- * alias x).  1 <= T <= max_tokens. */
+ * alias x).  1 <= T <= max_tokens.
+ * Execution (results are the same to the stated tolerance on every path):
+ * T <= 8 runs one persistent cooperative kernel when the shared-memory plan
+ * fits; larger T runs the router kernels and grouped expert GEMMs on the
+ * tensor cores (tcgen05 int8 MMA) when hidden and inter are multiples of
+ * 256, else CUDA-core grouped kernels.  Setting COLI_NO_TC=1 in the
+ * environment before coli_moe_create keeps the CUDA-core grouped kernels
+ * for that handle. */
 coli_status coli_moe_forward(coli_moe *m, const float *x, int T, float *out,
                              coli_stream_t stream);
 
