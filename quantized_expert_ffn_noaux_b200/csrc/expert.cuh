@@ -1367,7 +1367,11 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
                                             fa.G, fa.gk, k, fa.rsf, sm, pub ? fa.ws.idx + t * k : nullptr,
                                             pub ? fa.ws.w + t * k : nullptr, idx_s + t * k);
         }
-        cta_union_small<SyncConsumers>(lw, T, E, S, k, cnt, idx_s, reinterpret_cast<int *>(red));
+        if (MAXT == 1) {
+            if (warp == 0) warp_union_one(lw, E, S, k, idx_s);
+        } else {
+            cta_union_small<SyncConsumers>(lw, T, E, S, k, cnt, idx_s, reinterpret_cast<int *>(red));
+        }
         cp_async_wait_all();
         named_bar(1, 256);
         if (pub) {

@@ -276,6 +276,40 @@ __device__ void cta_select_token(const double *c_row, const double *s_row, int E
     Sync::sync();
 }
 
+// Batch-union tables of a single token, by one warp: the k selected experts
+// ascending (one pair each), then the shared experts -- the tables
+// cta_union_small builds for T = 1, without its scans over every expert.
+__device__ void warp_union_one(RouteWs ws, int E, int S, int k, const int *idx /*smem [k]*/) {
+    const int lane = threadIdx.x & 31;
+    for (int e = lane; e < E + S; e += 32) ws.act_of[e] = -1;
+    __syncwarp();
+    for (int j = lane; j < k; j += 32) {
+        const int e = idx[j];
+        int a = 0;
+        for (int i = 0; i < k; ++i) a += idx[i] < e;
+        ws.active[a] = e;
+        ws.off[a] = a;
+        ws.act_of[e] = a;
+        ws.pair_tok[a] = 0;
+        ws.pair_slot[a] = j;
+        ws.tok_pair[j] = a;
+    }
+    for (int i = lane; i < S; i += 32) {
+        const int a = k + i;
+        ws.active[a] = E + i;
+        ws.off[a] = a;
+        ws.act_of[E + i] = a;
+        ws.pair_tok[a] = 0;
+        ws.pair_slot[a] = k + i;
+        ws.tok_pair[k + i] = a;
+    }
+    if (lane == 0) {
+        ws.off[k + S] = k + S;
+        *ws.n_active = k + S;
+    }
+    __syncwarp();
+}
+
 // One CTA (256 threads) per token: cta_select_token.  With `do_union`, the
 // experts are also marked in the membership bitmap and the last CTA to finish
 // builds the batch-union tables.  Dynamic smem: select_smem_bytes(E, G).
