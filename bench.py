@@ -68,6 +68,22 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def over_ranks(value, op, device):
+    """`value` combined over every rank of the process group ("max" or "sum");
+    the value itself when there is no group or a single rank."""
+    dist = torch.distributed
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank_step, steps, world, ms_max):
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank_step * steps * world / (ms_max / 1e3)
+
+
 def sm_max_mhz():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -254,15 +270,9 @@ def run_coli(args, cfg, rank, world, device):
         launches_per_step = (qe.launch_count() - c0) / args.steps
     gpu_launches = int(round(launches_per_step * args.steps))
     bytes_timed = sum(bytes_per_step[s % L] for s in range(args.steps))
-    if world > 1:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-        tb = torch.tensor([float(bytes_timed)], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(tb)
-        bytes_timed = float(tb.item())
-    tokens = T * args.steps * world
-    value = tokens / (ms / 1e3)
+    ms = over_ranks(ms, "max", device)
+    bytes_timed = over_ranks(bytes_timed, "sum", device)
+    value = job_tokens_per_s(T, args.steps, world, ms)
     gbs = bytes_timed / (ms / 1e3) / 1e9
 
     # ---- per-kernel times (events on the launching stream), eager steps
@@ -341,10 +351,7 @@ def run_coli(args, cfg, rank, world, device):
         for s in range(n_e2e):
             layers[s % L].forward_host(xh[s % L], yh[s % L])
         e2e_s = time.perf_counter() - t0
-    if world > 1:
-        t = torch.tensor([e2e_s], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_s = float(t.item())
+    e2e_s = over_ranks(e2e_s, "max", device)
     e2e = {"value": round(T * n_e2e * world / e2e_s, 2), "unit": "tokens/s",
            "h2d_bytes_per_step": int(xh[0].numel() * 4), "d2h_bytes_per_step": int(yh[0].numel() * 4),
            "steps": n_e2e, "api": "coli_moe_forward_host (pinned host buffers, synchronous)"}
