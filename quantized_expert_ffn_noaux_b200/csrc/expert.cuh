@@ -876,6 +876,17 @@ __host__ __device__ inline DecodeSmem decode_smem(int T, int H, int I, int E, in
 }
 
 
+// One decision for all 8 consumer warps: whether the launch was aborted.
+// Every consumer warp calls it at the same point; one thread reads the flag
+// between two consumer barriers, so no warp leaves while another waits at a
+// later barrier for it.
+__device__ __forceinline__ bool consumers_aborted(volatile int *abort, int *flag_smem) {
+    named_bar(1, 256);
+    if (threadIdx.x == 0) *(volatile int *)flag_smem = *abort;
+    named_bar(1, 256);
+    return *(volatile int *)flag_smem != 0;
+}
+
 // P4 of the decode kernel: the consumer side of the down stages of this CTA's
 // output rows, one active expert after another.  VPL = vectors per lane of
 // the h activation (1, 2, 4: register-resident activation, loaded once per
@@ -1388,7 +1399,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         }
     }
     named_bar(2, DECODE_THREADS);        // tables ready: release producer and epilogue warp
-    if (*abort) return;
+    if (consumers_aborted(abort, flags + 1)) return;
 
     // P3: gate/up items; partials go to the epilogue warp through part_full /
     // part_free (two buffers)
@@ -1466,8 +1477,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         }
     }
     cp_async_wait_all();
-    named_bar(1, 256);
-    if (*abort) return;
+    if (consumers_aborted(abort, flags + 1)) return;
     // P4: down rows of every active expert as its h arrives, then the combine
     const int vpl = (VI % 32 == 0) ? VI / 32 : 0;
     DownLoop dl{lw.off, n_active, S, T, subs, ns, fa.down_rows, fa.rows_cap, r0, nrows, RBI, VI, I, rbI,
@@ -1478,8 +1488,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         case 4: ok = down_loop<BITS, 4, MAXT>(dl, rp) && ok; break;
         default: ok = down_loop<BITS, 0, MAXT>(dl, rp) && ok; break;
     }
-    named_bar(1, 256);
-    if (*abort) return;
+    if (consumers_aborted(abort, flags + 1)) return;
     const int slots = k + S;
     for (int q = tid; q < T * nrows; q += 256) {
         const int t = q / nrows, row = q % nrows;

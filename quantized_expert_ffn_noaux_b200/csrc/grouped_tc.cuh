@@ -61,6 +61,7 @@ struct TcBars {
     int abort;
     int n_items;
     int pad;
+    int pair_ok[16];   // gate/up epilogue pairs: each warp's ok, exchanged at the item's end
 };
 
 struct TcLayout {
@@ -588,9 +589,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
 #pragma unroll
                     for (int t = 0; t < NH; ++t) dst[(c0 + t) * 32 + lane] = (float)(acc[t] * sw);
                 }
-                const int bar_id = 1 + q + 4 * hh;
+                // the two warps of the pair decide together (either failing
+                // ends both, at the same item)
+                const int bar_id = 1 + q + 4 * hh, pid = 2 * (q + 4 * hh);
+                if (lane == 0) *(volatile int *)&tb->pair_ok[pid + m] = ok ? 1 : 0;
                 asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
-                if (m == 0 && ok && !*(volatile int *)&tb->abort) {
+                ok = *(volatile int *)&tb->pair_ok[pid] && *(volatile int *)&tb->pair_ok[pid + 1];
+                if (m == 0 && ok) {
                     const int nb = a.I / COLI_QBLK;
                     const int tend = min(c0 + NH, nt);
                     for (int t = c0; t < tend; ++t) {
