@@ -48,6 +48,8 @@ def lib():
         _LIB.oracle_route.argtypes = [vp, i64, i64, vp, vp, ci, ci, ci, ci, cf, vp, vp, vp, vp,
                                       vp, vp]
         _LIB.oracle_route.restype = ci
+        _LIB.oracle_swiglu.argtypes = [vp, vp, i64, vp]
+        _LIB.oracle_swiglu.restype = None
         _LIB.oracle_expert.argtypes = [i64, i64, ci, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         _LIB.oracle_expert.restype = ci
         _LIB.oracle_moe_forward.argtypes = [vp, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp,
@@ -144,6 +146,16 @@ def route(x, Wr, bias, top_k, n_group, topk_group, rsf):
         raise ValueError("oracle_route rejected E=%d G=%d gk=%d k=%d" % (E, n_group, topk_group,
                                                                         top_k))
     return dict(idx=idx, w=w, s=s, c=c, kmargin=km, gmargin=gm)
+
+
+def swiglu(g, u):
+    """SwiGLU of fp32 gate/up outputs -> h fp32 (same shape)."""
+    g = _c(g, np.float32).reshape(-1)
+    u = _c(u, np.float32).reshape(-1)
+    assert g.shape == u.shape
+    h = np.empty_like(g)
+    lib().oracle_swiglu(_p(g), _p(u), g.size, _p(h))
+    return h
 
 
 class QExpert:

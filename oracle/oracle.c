@@ -35,8 +35,10 @@
  *
  * Parity pins (tests/test_oracle_pins.py): hand-picked quantiser values,
  * pack/unpack identities, exact rational dots, brute-force routing
- * enumeration, routing invariants, the dense-mixture special case and an
- * exact single-expert case.  Layer-level values are not printed by the pages.
+ * enumeration, routing invariants, the dense-mixture special case, an exact
+ * single-expert case, and SwiGLU values and a whole unsaturated expert
+ * derived by exact arithmetic (tests/golden/make_swiglu.py).  Layer-level
+ * values are not printed by the pages.
  */
 #include <math.h>
 #include <stdint.h>
@@ -336,6 +338,18 @@ typedef struct {
     const float *scales;
 } oracle_qmat;
 
+/* The SwiGLU activation of one expert's gate and up outputs:
+ *   h[i] = (float)( SiLU(g[i]) * u[i] ),  SiLU(g) = g * sigmoid(g) = g / (1 + exp(-g)),
+ * evaluated in fp64 from the fp32 g, u and rounded once to fp32.  The sigmoid
+ * gates the gate projection g, never the up projection u. */
+void oracle_swiglu(const float *g, const float *u, int64_t n, float *h)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        double gd = (double)g[i];
+        h[i] = (float)((gd / (1.0 + exp(-gd))) * (double)u[i]);
+    }
+}
+
 static void expert_token(int64_t H, int64_t I, int bits, const oracle_qmat *gate,
                          const oracle_qmat *up, const oracle_qmat *down, const int8_t *xq,
                          const float *xd, const int8_t *hq_in, const float *hd_in,
@@ -344,10 +358,7 @@ static void expert_token(int64_t H, int64_t I, int bits, const oracle_qmat *gate
     float *g = scratch, *u = scratch + I, *h = scratch + 2 * I;
     oracle_int_dot(gate->codes, gate->scales, bits, I, H, xq, xd, g);
     oracle_int_dot(up->codes, up->scales, bits, I, H, xq, xd, u);
-    for (int64_t i = 0; i < I; ++i) {
-        double gd = (double)g[i];
-        h[i] = (float)((gd / (1.0 + exp(-gd))) * (double)u[i]);
-    }
+    oracle_swiglu(g, u, I, h);
     const int8_t *hq;
     const float *hd;
     if (hq_in && hd_in) {

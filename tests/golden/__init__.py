@@ -65,4 +65,37 @@ def single_expert_y():
     return np.array(ys, np.float32)
 
 
-__all__ = ["q8_blocks", "weight_rows", "single_expert_y", "Fraction"]
+def swiglu_cases():
+    """[(g, u, h)] fp32 triples from swiglu_cases.txt."""
+    out = []
+    for ln in _lines("swiglu_cases.txt"):
+        g, u, h = (np.float32(float(v)) for v in ln.split("|"))
+        out.append((g, u, h))
+    return out
+
+
+def swiglu_expert():
+    """The one-expert case of swiglu_expert.txt as a dict of numpy arrays:
+    x [1][32], gate/up [32][32], down [32][32] fp32; g, u, h [32] fp32;
+    hq [32] int8; hd fp32 scalar; y [32] fp32; rsf float."""
+    rows = {"gate": {}, "up": {}, "down": {}}
+    d = {}
+    for ln in _lines("swiglu_expert.txt"):
+        key, val = ln.split(":", 1)
+        parts = key.split()
+        if parts[0] in rows:
+            rows[parts[0]][int(parts[1])] = [float(v) for v in val.split()]
+        else:
+            d[key.strip()] = val.split()
+    out = {name: np.array([m[r] for r in range(len(m))], np.float32) for name, m in rows.items()}
+    out["x"] = np.array([[float(v) for v in d["x"]]], np.float32)
+    for k in ("g", "u", "h", "y"):
+        out[k] = np.array([float(v) for v in d[k]], np.float32)
+    out["hq"] = np.array([int(v) for v in d["hq"]], np.int8)
+    out["hd"] = np.float32(float(d["hd"][0]))
+    out["rsf"] = float(d["rsf"][0])
+    return out
+
+
+__all__ = ["q8_blocks", "weight_rows", "single_expert_y", "swiglu_cases", "swiglu_expert",
+           "Fraction"]

@@ -5,6 +5,8 @@ The CUDA side quantises its weights with its own kernel; the oracle quantises
 host copies of the same fp32 tensors with its own C code.  Weight codes are
 compared bit for bit wherever both sides have them.
 """
+import itertools
+
 import numpy as np
 import torch
 
@@ -74,20 +76,67 @@ def decidable(route_res, t):
     return route_res["kmargin"][t] > MARGIN and route_res["gmargin"][t] > MARGIN
 
 
-def check_route(gpu_idx, gpu_w, ref, tokens=None):
+def _group_scores(c, G):
+    """Sum of the two largest choice scores of each group (one if a group has
+    a single expert)."""
+    per = c.shape[0] // G
+    cg = np.sort(c.reshape(G, per), axis=1)[:, ::-1]
+    return cg[:, 0] + (cg[:, 1] if per > 1 else 0.0)
+
+
+def valid_tie_choice(sel, c, G, gk, k, margin=MARGIN):
+    """Whether the expert set `sel` is a correct selection for choice scores
+    `c` once every comparison closer than `margin` may go either way: some
+    set K of gk groups holds every group whose score is clearly above the
+    gk-th and none clearly below it, `sel` is k distinct experts of K's
+    groups, and every expert of K left out of `sel` is not clearly above any
+    expert in it (a valid alternative of the group-limited top-k)."""
+    sel = [int(e) for e in sel]
+    E = c.shape[0]
+    if len(sel) != k or len(set(sel)) != k or min(sel) < 0 or max(sel) >= E:
+        return False
+    per = E // G
+    gs = _group_scores(c, G)
+    theta = np.sort(gs)[::-1][gk - 1]
+    must = [g for g in range(G) if gs[g] > theta + margin]
+    may = [g for g in range(G) if abs(gs[g] - theta) <= margin]
+    if not set(e // per for e in sel) <= set(must) | set(may):
+        return False
+    for fill in itertools.combinations(may, gk - len(must)):
+        kept = set(must) | set(fill)
+        if not all(e // per in kept for e in sel):
+            continue
+        rest = [e for e in range(E) if e // per in kept and e not in sel]
+        lo = min(c[e] for e in sel)
+        if all(c[e] <= lo + margin for e in rest):
+            return True
+    return False
+
+
+def check_route(gpu_idx, gpu_w, ref, tokens=None, G=None, gk=None, rsf=None):
     """Bit-exact idx for decidable tokens (as sets, order where the c gap is
-    clear); weights within 1e-6 relative.  Returns the undecidable tokens."""
+    clear); weights within 1e-6 relative of the renormalised sigmoid scores of
+    the chosen set.  Undecidable tokens (a routing margin within 1e-5) must
+    carry a valid tie alternative (valid_tie_choice) sorted by descending c up
+    to the margin.  Returns the undecidable tokens."""
     gpu_idx = np.asarray(gpu_idx)
     gpu_w = np.asarray(gpu_w)
     tokens = range(gpu_idx.shape[0]) if tokens is None else tokens
     loose = []
     for i, t in enumerate(tokens):
+        gi, ri = gpu_idx[i], ref["idx"][t]
+        c = ref["c"][t]
         if not decidable(ref, t):
+            assert G is not None and gk is not None, "check_route needs G, gk for near ties"
+            assert valid_tie_choice(gi, c, G, gk, len(ri)), (t, gi, ri)
+            for j in range(len(gi) - 1):
+                assert c[gi[j]] >= c[gi[j + 1]] - MARGIN, (t, j, gi)
+            s = ref["s"][t][gi]
+            scale = float(ref["w"][t].astype(np.float64).sum()) if rsf is None else rsf
+            np.testing.assert_allclose(gpu_w[i], s / s.sum() * scale, rtol=1e-6)
             loose.append(i)
             continue
-        gi, ri = gpu_idx[i], ref["idx"][t]
         assert set(gi.tolist()) == set(ri.tolist()), (t, gi, ri)
-        c = ref["c"][t]
         for j in range(len(ri) - 1):
             if c[ri[j]] - c[ri[j + 1]] > MARGIN:
                 assert gi[j] == ri[j], (t, j, gi, ri)
@@ -121,10 +170,12 @@ def compare_forward(gl, x_dev, tokens=None, check_h=True):
     probe = oracle.Layer(synth.layer_cfg(gl.cfg), gl.Wr.cpu().numpy(), gl.bias.cpu().numpy(),
                          [None] * (gl.cfg["n_routed"] + gl.cfg["n_shared"]))
     ref_route = probe.route(x_host)
-    loose = check_route(idx, w, ref_route)
+    loose = check_route(idx, w, ref_route, G=gl.cfg["n_group"], gk=gl.cfg["topk_group"],
+                        rsf=gl.cfg["routed_scaling_factor"])
     need = set(idx.reshape(-1).tolist()) | set(ref_route["idx"].reshape(-1).tolist())
     layer = gl.oracle_layer(need)
-    # undecidable tokens: the oracle re-runs with the CUDA side's (valid) choice
+    # undecidable tokens: the oracle re-runs with the CUDA side's choice, which
+    # check_route has confirmed to be a valid tie alternative
     idx_in = ref_route["idx"].copy()
     for i in loose:
         idx_in[i] = idx[i]

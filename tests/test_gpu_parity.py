@@ -78,7 +78,8 @@ def test_router_glm52_shape(T):
     idx, w = h.router(x)
     ref = oracle.route(x.cpu().numpy(), W.cpu().numpy(), b.cpu().numpy(), cfg["top_k"],
                        cfg["n_group"], cfg["topk_group"], cfg["routed_scaling_factor"])
-    loose = check_route(idx.cpu().numpy(), w.cpu().numpy(), ref)
+    loose = check_route(idx.cpu().numpy(), w.cpu().numpy(), ref, G=cfg["n_group"],
+                        gk=cfg["topk_group"], rsf=cfg["routed_scaling_factor"])
     assert len(loose) <= max(1, T // 50)
     h.close()
 

@@ -304,6 +304,59 @@ def test_single_expert_hand_computed():
     assert res["hd"][0, 0, 0] == np.float32(381.0)
 
 
+def test_swiglu_hand_values():
+    """h = SiLU(g) * u against its exact value rounded once to fp32
+    (tests/golden/make_swiglu.py), for |g| in [0.1, 4] of both signs, g != u,
+    and the zero and saturated cases."""
+    cases = golden.swiglu_cases()
+    g = np.array([c[0] for c in cases], np.float32)
+    u = np.array([c[1] for c in cases], np.float32)
+    h = np.array([c[2] for c in cases], np.float32)
+    np.testing.assert_array_equal(oracle.swiglu(g, u), h)
+
+
+def test_swiglu_fixture_separates_plausible_mistakes():
+    """The fixture has teeth: dropping the sigmoid, gating u instead of g,
+    ReLU in place of SiLU and sigmoid(+g) each disagree with it in most of the
+    unsaturated cases (so any of them in the oracle fails the pin above)."""
+    cases = [c for c in golden.swiglu_cases() if 0.1 <= abs(float(c[0])) <= 4.0
+             and float(c[1]) != 0.0]
+    assert len(cases) >= 40
+    g = np.array([c[0] for c in cases], np.float64)
+    u = np.array([c[1] for c in cases], np.float64)
+    h = np.array([c[2] for c in cases], np.float32)
+    sig = lambda v: 1.0 / (1.0 + np.exp(-v))  # noqa: E731
+    wrong = {
+        "no sigmoid": g * u,
+        "SiLU of u": u * sig(u) * g,
+        "ReLU": np.maximum(g, 0.0) * u,
+        "sigmoid(+g)": g / (1.0 + np.exp(g)) * u,
+    }
+    for name, v in wrong.items():
+        assert np.mean(v.astype(np.float32) != h) > 0.9, name
+
+
+def test_swiglu_expert_exact():
+    """One int4 expert whose g and u are exact fp32 values with |g| < 4:
+    the oracle's g, u, Q8_0(h) codes and scale and output y equal the values
+    make_swiglu.py derived by exact arithmetic."""
+    ex = golden.swiglu_expert()
+    H = I = 32
+    q = oracle.QExpert.quantise(ex["gate"], ex["up"], ex["down"], 4)
+    xq, xd = oracle.quant_q8(ex["x"])
+    np.testing.assert_array_equal(oracle.int_dot(*q.gate, 4, H, xq, xd), ex["g"])
+    np.testing.assert_array_equal(oracle.int_dot(*q.up, 4, H, xq, xd), ex["u"])
+    e, hq, hd = oracle.expert(H, I, 4, q, xq, xd)
+    np.testing.assert_array_equal(hq, ex["hq"])
+    assert hd[0] == ex["hd"]
+    cfg = _cfg(hidden=H, inter=I, n_routed=1, n_shared=0, top_k=1,
+               routed_scaling_factor=ex["rsf"])
+    layer = oracle.Layer(cfg, np.zeros((1, H), np.float32), np.zeros(1, np.float32), [q])
+    res = layer.forward(ex["x"])
+    np.testing.assert_array_equal(res["hq"][0, 0], ex["hq"])
+    np.testing.assert_array_equal(res["out"][0], ex["y"])
+
+
 def test_dense_mixture_when_k_equals_E():
     """top_k = E with one group: every expert is used with weight
     rsf * s_i / sum(s), so y = e_shared + rsf * sum_i (s_i / sum s) e_i."""
