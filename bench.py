@@ -53,7 +53,8 @@ def parse():
                    help="override the routed expert count (smaller layers for profiling)")
     p.add_argument("--e2e-steps", type=int, default=2000)
     p.add_argument("--profile-steps", type=int, default=400)
-    p.add_argument("--cpu-sample-tokens", type=int, default=8)
+    p.add_argument("--cpu-sample-tokens", type=int, default=None,
+                   help="tokens in the CPU-baseline sample (default: one per host thread)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-graph", action="store_true")
     return p.parse_args()
@@ -388,9 +389,12 @@ def oracle_layer_for(cfg, Wr, bias, needed, fp32_fn, threads):
 
 
 def cpu_baseline(cfg, layer0, x0, n_tok, device):
-    """The oracle on this host's cores: n_tok tokens of the workload (layer 0)."""
+    """The oracle on this host's cores: n_tok tokens of the workload (layer 0),
+    one token per OpenMP thread (the oracle splits tokens over threads and
+    nothing finer), plus one token on a single thread."""
     import oracle
     threads = os.cpu_count() or 1
+    n_tok = threads if n_tok is None else n_tok
     W, b = synth.router(cfg, device=device, layer=0)
     Wr, bias = W.cpu().numpy(), b.cpu().numpy()
     x = synth.tokens(cfg, T=n_tok, device=device, layer=0, stream=10**6).cpu().numpy()
@@ -402,9 +406,15 @@ def cpu_baseline(cfg, layer0, x0, n_tok, device):
     t0 = time.perf_counter()
     lay.forward(x, nthreads=threads)
     dt = time.perf_counter() - t0
-    return {"value": round(n_tok / dt, 4), "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": "%d tokens of %s (layer 0), one oracle forward, %d OpenMP threads over "
-                      "tokens, %.1f s" % (n_tok, cfg["name"], threads, dt)}
+    t0 = time.perf_counter()
+    lay.forward(x[:1], nthreads=1)
+    dt1 = time.perf_counter() - t0
+    used = min(threads, n_tok)
+    return {"value": round(n_tok / dt, 4), "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "single_thread": {"value": round(1.0 / dt1, 4), "unit": "tokens/s", "cores": 1},
+            "sample": "%d tokens of %s (layer 0) in one oracle forward on %d OpenMP threads, "
+                      "one token per thread, %.1f s; single thread: 1 token, %.2f s" % (
+                          n_tok, cfg["name"], used, dt, dt1)}
 
 
 # ------------------------------------------------------------- reference arm
@@ -457,16 +467,18 @@ def run_reference(args, cfg):
         one(args.warmup + i)
     dt = time.perf_counter() - t0
     value = T * args.steps * (m / slots) / dt
-    sample = ("each step: one %d-token batch of %s through the oracle (%s), %d threads"
+    used = 1 if m != slots else min(threads, T)  # OpenMP splits tokens, nothing finer
+    sample = ("each step: one %d-token batch of %s through the oracle (%s); the oracle splits "
+              "tokens over OpenMP threads, so %d of %d host threads work"
               % (T, cfg["name"], "all %d expert slots" % slots if m == slots else
                  "%d of %d expert slots per token, counted as %d/%d of a batch" % (m, slots, m, slots),
-                 threads))
+                 used, threads))
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": {"workload": cfg["name"], "tokens_per_step": T, "bits": cfg["bits"]},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}

@@ -419,6 +419,8 @@ struct PipePlan {
     int grid = 0;
     int rows_cap = 0;      // down: rows per CTA (max)
     int amax = 0, pmax = 0;
+    int nh = 0, h_alias = 0, ptr_smem = 0;  // decode kernel: h slots, their placement, pointer table
+    int down_span = 1;                       // ring slots per down stage
 };
 
 int ring_stages(size_t fixed, size_t stage) {
@@ -434,12 +436,39 @@ PipePlan plan_decode(const coli_moe *m, int T) {
     p.pmax = T * (c.top_k + c.n_shared);
     p.rows_cap = (c.hidden + p.grid - 1) / p.grid;
     const int RBI = c.inter * c.wfmt / 8;
-    // at most 8 rows per consumer warp in a down stage
-    p.stage_rows = std::max(1, std::min(std::min(p.rows_cap, PIPE_STAGE_MAX / RBI), 8 * PIPE_CONSUMERS));
-    const size_t fixed = decode_smem(T, c.hidden, c.inter, c.n_routed, c.n_shared, c.n_group,
-                                     c.top_k, p.pmax, g.slices, p.rows_cap, 0).total;
-    p.ns = ring_stages(fixed, PIPE_STAGE_MAX);
-    p.smem = fixed + (size_t)p.ns * PIPE_STAGE_MAX;
+    p.amax = std::min(c.n_routed, T * c.top_k) + c.n_shared;
+    auto fixed = [&](int nh, int alias, int ptrs) {
+        return decode_smem(T, c.hidden, c.inter, c.n_routed, c.n_shared, c.n_group, c.top_k,
+                           p.pmax, g.slices, p.rows_cap, 0, nh, alias, ptrs).total;
+    };
+    // h slots of their own (filled as soon as each expert's h is complete) as
+    // many as fit beside a ring of at least 4 stages; else two slots in the
+    // x records' space (filled after the gate/up items)
+    p.ptr_smem = c.n_routed + c.n_shared <= DECODE_PTR_SMEM_MAX ? 1 : 0;
+    p.nh = 2;
+    p.h_alias = 1;
+    for (int nh = std::min(p.amax, DECODE_MAX_HSLOTS); nh >= 2; --nh) {
+        if (ring_stages(fixed(nh, 0, p.ptr_smem), PIPE_STAGE_MAX) >= 4) {
+            p.nh = nh;
+            p.h_alias = 0;
+            break;
+        }
+    }
+    if (p.h_alias && ring_stages(fixed(2, 1, p.ptr_smem), PIPE_STAGE_MAX) < 3) p.ptr_smem = 0;
+    const size_t f = fixed(p.nh, p.h_alias, p.ptr_smem);
+    p.ns = ring_stages(f, PIPE_STAGE_MAX);
+    // Down stages: a CTA's rows of one expert are fetched in as few bulk
+    // copies as possible -- DRAM serves one copy per slice far better than
+    // the slice split over several stages -- so with an even ring a down
+    // stage takes two adjacent slots.  At most 8 rows per consumer warp.
+    p.down_span = p.ns >= 4 ? 2 : 1;
+    if (p.down_span == 2) p.ns &= ~1;
+    const int cap_rows = p.down_span * PIPE_STAGE_MAX / RBI;
+    const int want = (p.rows_cap + PIPE_CONSUMERS - 1) / PIPE_CONSUMERS * PIPE_CONSUMERS;
+    int rows = std::min(want, cap_rows >= PIPE_CONSUMERS ? cap_rows / PIPE_CONSUMERS * PIPE_CONSUMERS
+                                                         : cap_rows);
+    p.stage_rows = std::max(1, std::min(rows, 8 * PIPE_CONSUMERS));
+    p.smem = f + (size_t)p.ns * PIPE_STAGE_MAX;
     return p;
 }
 
@@ -539,6 +568,10 @@ coli_status launch_small_path(coli_moe *m, const float *x, int T, float *out, cu
     fa.pmax = p.pmax;
     fa.rows_cap = p.rows_cap;
     fa.down_rows = p.stage_rows;
+    fa.down_span = p.down_span;
+    fa.nh = p.nh;
+    fa.h_alias = p.h_alias;
+    fa.ptr_smem = p.ptr_smem;
     Launch L(m, s, "moe_decode");
     cudaError_t e = launch_coop(kern, dim3(p.grid), dim3(DECODE_THREADS), p.smem, s, fa);
     if (e != cudaSuccess) return cuda_fail(e, "moe_decode launch");

@@ -267,6 +267,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking probe of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait that yields the issue slots while it waits: for threads whose
 // wait is long and whose wake-up latency matters little (the producer thread
 // waiting for a free ring slot, the epilogue warp waiting for partials), so
@@ -339,6 +351,20 @@ __device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, uint32
 
 __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Release-ordered add at GPU scope: this thread's earlier writes (and those
+// ordered before them, e.g. by a warp barrier) are visible to any thread that
+// acquires the counter value this add produces.
+__device__ __forceinline__ void red_release_add(int *p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Arrive on `bar` once every cp.async this thread issued so far has landed;
+// the barrier's expected count includes these arrivals (.noinc).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
 }
 
 // Programmatic dependent launch: wait for the preceding grid's completion and

@@ -398,8 +398,9 @@ __global__ void __launch_bounds__(256) k_down_combine(RouteWs ws,
 // returns.
 constexpr int PIPE_CONSUMERS = 8;
 constexpr int PIPE_THREADS = 32 * (PIPE_CONSUMERS + 1);
-// the decode kernel adds an epilogue warp: 8 consumers, producer, epilogue
-constexpr int DECODE_THREADS = 32 * (PIPE_CONSUMERS + 2);
+// the decode kernel adds an epilogue warp and an h-fetch warp: 8 consumers,
+// producer, epilogue, h fetch
+constexpr int DECODE_THREADS = 32 * (PIPE_CONSUMERS + 3);
 constexpr int PIPE_STAGE_MAX = 24 * 1024;  // bytes of weights per ring stage (at most)
 constexpr int PIPE_MAX_STAGES = 8;
 constexpr int PIPE_MAX_TOK = 8;            // tokens per expert on the few-token path
@@ -602,14 +603,28 @@ struct RingPos {
     }
 };
 
-// The ring as the consumers see it.
+// The ring as the consumers see it.  A down stage may span two adjacent
+// slots (one bulk copy of up to twice the slot size, starting on an even
+// slot); the second slot's full phase completes without data.
 struct RingView {
     const uint8_t *ring;
     PipeBars *bars;
     int ns;
     int *err;
     volatile int *abort;
+    int span = 1;
 };
+
+// Consumer side of releasing one (possibly two-slot) stage: every lane has
+// finished reading it.
+__device__ __forceinline__ void release_stage(PipeBars *bars, RingPos &rp, int ns, int span) {
+    const int lane = threadIdx.x & 31;
+    __syncwarp();
+    for (int z = 0; z < span; ++z) {
+        if (lane == 0) mbar_arrive(&bars->empty[rp.slot]);
+        rp.next(ns);
+    }
+}
 
 // Consumer side of one whole gate/up item on the fast geometry (SL slices of
 // the row, R = 16 / SL rows a stage, 2 SL stages a matrix): a warp keeps the
@@ -664,6 +679,11 @@ __device__ __forceinline__ void cp_async_wait_all() {
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.relaxed.gpu.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
 
@@ -753,8 +773,9 @@ __device__ __forceinline__ bool down_expert_deferred(const RingView &rv, RingPos
                                                      const LaneAct<BITS, VPL> &act, int p, float *ebuf,
                                                      int rows_cap) {
     constexpr int N = RPW * SUBS;
-    constexpr int U = N <= 4 ? 4 : 8;
-    constexpr int SHIFT = U == 4 ? 3 : 2;
+    static_assert(N <= 16, "at most 16 deferred rows per warp");
+    constexpr int U = N <= 4 ? 4 : (N <= 8 ? 8 : 16);
+    constexpr int SHIFT = U == 4 ? 3 : (U == 8 ? 2 : 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     double acc[U];
 #pragma unroll
@@ -773,9 +794,7 @@ __device__ __forceinline__ bool down_expert_deferred(const RingView &rv, RingPos
             acc[sb * RPW + i] =
                 row < nr ? act.dot(reinterpret_cast<const uint4 *>(stage + (size_t)row * RB), 0) : 0.0;
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&rv.bars->empty[rp.slot]);
-        rp.next(rv.ns);
+        release_stage(rv.bars, rp, rv.ns, rv.span);
     }
     const double tot = warp_sum_rows<U>(acc);
     const int j = lane >> SHIFT, sb = j / RPW, i = j - sb * RPW;
@@ -836,14 +855,25 @@ struct DecodeArgs {
     int ns, pmax;
     int rows_cap;       // output rows per CTA (max) in P4
     int down_rows;      // down rows per stage
+    int down_span;      // ring slots per down stage (1, or 2: one copy across two adjacent slots)
+    int nh;             // shared slots for the h records of active experts (<= DECODE_MAX_HSLOTS)
+    int h_alias;        // 1: the slots reuse the x records' space, so they fill only after P3
+    int ptr_smem;       // 1: every expert's code pointers are staged in shared memory in P1
 };
 
+constexpr int DECODE_MAX_HSLOTS = 16;
+// every expert's gate/up/down code pointers and down scales pointer staged in
+// shared memory while routing runs, when E + S is at most this
+constexpr int DECODE_PTR_SMEM_MAX = 320;
+
 struct DecodeSmem {
-    size_t select, idxw, cnt, red, tables, act, ebuf, part, dscale, eptr, ring, total;
+    size_t select, idxw, cnt, red, tables, act, hslot, hbar, eptrs, ebuf, part, dscale, eptr, ring,
+        total;
 };
 
 __host__ __device__ inline DecodeSmem decode_smem(int T, int H, int I, int E, int S, int G, int k,
-                                                  int pmax, int slices, int rows_cap, int ns) {
+                                                  int pmax, int slices, int rows_cap, int ns,
+                                                  int nh, int h_alias, int ptr_smem) {
     DecodeSmem d;
     size_t o = pipe_hdr_bytes();
     d.ring = o;
@@ -858,9 +888,20 @@ __host__ __device__ inline DecodeSmem decode_smem(int T, int H, int I, int E, in
     o += align128((size_t)2 * 8 * PIPE_MAX_TOK * 8);
     d.tables = o;
     o += align128((size_t)(3 * (E + S) + 1 + 3 * pmax + 4) * 4);
-    d.act = o;
-    const size_t xa = (size_t)T * rec_bytes(H), ha = (size_t)2 * T * rec_bytes(I);
-    o += align128(xa > ha ? xa : ha);
+    const size_t xa = (size_t)T * rec_bytes(H), ha = (size_t)nh * T * rec_bytes(I);
+    d.act = o;                            // Q8_0(x) records of the T tokens
+    if (h_alias) {                        // nh slots of T h records each, in the same space
+        d.hslot = o;
+        o += align128(xa > ha ? xa : ha);
+    } else {
+        o += align128(xa);
+        d.hslot = o;
+        o += align128(ha);
+    }
+    d.hbar = o;                           // h_full[nh], h_empty[nh], x_free
+    o += align128((size_t)(2 * nh + 1) * 8);
+    d.eptrs = o;                          // 4 pointers per expert (ptr_smem only)
+    o += ptr_smem ? align128((size_t)(E + S) * 4 * sizeof(void *)) : 0;
     d.ebuf = o;
     o += align128((size_t)pmax * rows_cap * 4);
     d.part = o;
@@ -895,19 +936,19 @@ __device__ __forceinline__ bool consumers_aborted(volatile int *abort, int *flag
 struct EpiBars {
     uint64_t part_full[2];   // the 8 consumer warps finished an item's partials
     uint64_t part_free[2];   // the epilogue warp finished reading them
-    uint64_t h_full[2];      // an expert's h records are in its shared slot
-    uint64_t h_empty[2];     // the 8 consumer warps are done with that slot
 };
 
 struct DownLoop {
     const int *off;
-    int n_active, S, T, subs, ns, down_rows, rows_cap, r0, nrows, RBI, VI, I, rbI;
+    int n_active, S, T, subs, ns, down_rows, rows_cap, r0, nrows, RBI, VI, I, rbI, span;
     const uint8_t *ring;
     const float *dscale;
-    const uint8_t *acts;     // two slots of T h records each, filled by the epilogue warp
+    const uint8_t *hslots;   // nh slots of T h records each, filled by the epilogue warp
+    int nh;
+    uint64_t *hfull;         // [nh] an expert's h records are in its slot (32 cp.async arrivals)
+    uint64_t *hempty;        // [nh] the 8 consumer warps are done with that slot
     float *ebuf;
     PipeBars *bars;
-    EpiBars *ebars;
     volatile int *abort;
     int *err;
 };
@@ -925,10 +966,11 @@ __device__ __forceinline__ bool down_loop(const DownLoop &d, RingPos &rp) {
     for (int q = 0; q < d.n_active; ++q) {
         const int a = down_slot(q, d.n_active, d.S);
         const int p0 = d.off[a], ne = d.off[a + 1] - p0;
-        // this expert's h records: slot q & 1, filled once all its gate/up
+        // this expert's h records: slot q % nh, filled once all its gate/up
         // items (any CTA's) are written
-        const uint8_t *recs = d.acts + (size_t)(q & 1) * d.T * d.rbI;
-        if (!mbar_wait(&d.ebars->h_full[q & 1], (uint32_t)(q >> 1) & 1u, d.err)) {
+        const int hs = q % d.nh;
+        const uint8_t *recs = d.hslots + (size_t)hs * d.T * d.rbI;
+        if (!mbar_wait(&d.hfull[hs], (uint32_t)((q / d.nh) & 1), d.err)) {
             *d.abort = 1;
             return false;
         }
@@ -940,16 +982,22 @@ __device__ __forceinline__ bool down_loop(const DownLoop &d, RingPos &rp) {
                 act.load(recs, d.I, d.VI, 0);
                 // whole expert at once where the stage geometry allows
                 const float *sc_a = d.dscale + a * (d.rows_cap + 4);
-                const RingView rv{d.ring, d.bars, d.ns, d.err, d.abort};
+                const RingView rv{d.ring, d.bars, d.ns, d.err, d.abort, d.span};
                 if (d.down_rows == 8 * rpw) {
-                    if (rpw == 3 && d.subs == 2)
-                        done = down_expert_deferred<BITS, VPL, 3, 2>(rv, rp, d.RBI, d.nrows, sc_a, act, p0, d.ebuf, d.rows_cap);
-                    else if (rpw == 4 && d.subs == 2)
-                        done = down_expert_deferred<BITS, VPL, 4, 2>(rv, rp, d.RBI, d.nrows, sc_a, act, p0, d.ebuf, d.rows_cap);
-                    else if (rpw == 2 && d.subs <= 4 && d.subs >= 3)
-                        done = d.subs == 3
-                                   ? down_expert_deferred<BITS, VPL, 2, 3>(rv, rp, d.RBI, d.nrows, sc_a, act, p0, d.ebuf, d.rows_cap)
-                                   : down_expert_deferred<BITS, VPL, 2, 4>(rv, rp, d.RBI, d.nrows, sc_a, act, p0, d.ebuf, d.rows_cap);
+#define COLI_DEFER(R, SB) done = down_expert_deferred<BITS, VPL, R, SB>(rv, rp, d.RBI, d.nrows, sc_a, act, p0, d.ebuf, d.rows_cap)
+                    if (rpw == 6 && d.subs == 1) COLI_DEFER(6, 1);
+                    else if (rpw == 6 && d.subs == 2) COLI_DEFER(6, 2);
+                    else if (rpw == 4 && d.subs == 1) COLI_DEFER(4, 1);
+                    else if (rpw == 2 && d.subs == 1) COLI_DEFER(2, 1);
+                    else if (rpw == 3 && d.subs == 1) COLI_DEFER(3, 1);
+                    else if (rpw == 3 && d.subs == 2) COLI_DEFER(3, 2);
+                    else if (rpw == 3 && d.subs == 3) COLI_DEFER(3, 3);
+                    else if (rpw == 3 && d.subs == 4) COLI_DEFER(3, 4);
+                    else if (rpw == 4 && d.subs == 2) COLI_DEFER(4, 2);
+                    else if (rpw == 2 && d.subs == 2) COLI_DEFER(2, 2);
+                    else if (rpw == 2 && d.subs == 3) COLI_DEFER(2, 3);
+                    else if (rpw == 2 && d.subs == 4) COLI_DEFER(2, 4);
+#undef COLI_DEFER
                 }
                 if (done == 0) return false;
             }
@@ -990,14 +1038,12 @@ __device__ __forceinline__ bool down_loop(const DownLoop &d, RingPos &rp) {
                     }
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&d.bars->empty[rp.slot]);
-            rp.next(d.ns);
+            release_stage(d.bars, rp, d.ns, d.span);
         }
         if (!expert_ok) return false;
         // the slot may be refilled
         __syncwarp();
-        if (lane == 0) mbar_arrive(&d.ebars->h_empty[q & 1]);
+        if (lane == 0) mbar_arrive(&d.hempty[hs]);
     }
     return true;
 }
@@ -1040,7 +1086,8 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
     const int R = geo.R, slices = geo.slices, spm = 32 / R, steps = 2 * spm;
     const int nchunk = I / 32, rbH = rec_bytes(H), rbI = rec_bytes(I), nbH = H / COLI_QBLK;
     const int ns = fa.ns, G = gridDim.x;
-    const DecodeSmem L = decode_smem(T, H, I, E, S, fa.G, k, fa.pmax, slices, fa.rows_cap, ns);
+    const DecodeSmem L = decode_smem(T, H, I, E, S, fa.G, k, fa.pmax, slices, fa.rows_cap, ns,
+                                     fa.nh, fa.h_alias, fa.ptr_smem);
     uint8_t *ring = smem + L.ring;
     SelectSmem sm = carve_select(smem + L.select, E, fa.G);
     int *idx_s = reinterpret_cast<int *>(smem + L.idxw);
@@ -1056,7 +1103,14 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
     lw.tok_pair = lw.pair_slot + fa.pmax;
     lw.n_active = lw.tok_pair + fa.pmax;
     int *flags = lw.n_active + 1;
-    uint8_t *acts = smem + L.act;       // x records in P2/P3, h records in P4
+    uint8_t *acts = smem + L.act;       // x records (P2, P3)
+    uint8_t *hslots = smem + L.hslot;   // h records of active experts (P3, P4)
+    uint64_t *hfull = reinterpret_cast<uint64_t *>(smem + L.hbar);
+    uint64_t *hempty = hfull + fa.nh;
+    uint64_t *xfree = hempty + fa.nh;   // the consumers are done with the x records (after P3)
+    // gate, up, down code pointers and the down scales pointer of every expert
+    // (ptr_smem), staged by the epilogue warp while routing runs
+    const void **eptrs = reinterpret_cast<const void **>(smem + L.eptrs);
     float *ebuf = reinterpret_cast<float *>(smem + L.ebuf);
     double *part = reinterpret_cast<double *>(smem + L.part);
     float *dscale = reinterpret_cast<float *>(smem + L.dscale);   // [active][rows_cap + 4]
@@ -1071,9 +1125,12 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&ebars->part_full[i], PIPE_CONSUMERS);
             mbar_init(&ebars->part_free[i], 1);
-            mbar_init(&ebars->h_full[i], 1);
-            mbar_init(&ebars->h_empty[i], PIPE_CONSUMERS);
         }
+        for (int i = 0; i < fa.nh; ++i) {
+            mbar_init(&hfull[i], 32);   // one cp.async completion arrival per epilogue lane
+            mbar_init(&hempty[i], PIPE_CONSUMERS);
+        }
+        mbar_init(xfree, PIPE_CONSUMERS);
     }
     pipe_init(bars, ns);
     __syncthreads();
@@ -1100,7 +1157,10 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         RingPos rp;
         const uint64_t pol = l2_evict_first_policy();
         int issued = 0;
-        // let the router-weight loads enter the memory queues first
+        // routing goes first: the consumers release this barrier once the
+        // selection's scores are in shared memory, so neither the router
+        // weights nor the grid barrier nor those loads queue behind the
+        // shared expert's bulk copies in the memory system
         asm volatile("bar.sync 4, %0;" ::"r"(32 * (PIPE_CONSUMERS + 1)) : "memory");
         int q_ld = -1;
         const uint8_t *sh_gate = nullptr, *sh_up = nullptr;
@@ -1120,9 +1180,21 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
             rp.next(ns);
             cur.next(1 << 30, steps, subs);
         }
-        if (lane == 0)  // warm L2 with the shared experts' down rows of this CTA
+        if (lane == 0) {
+            // the rest of this CTA's shared gate/up stages (beyond the ring)
+            // into L2, then the shared experts' down rows of this CTA
+            StageCursor c2 = cur;
+            for (int n = 0; n < steps && item_of(c2.j) < n_shared_items; ++n) {
+                const int item = item_of(c2.j);
+                const int q = item / nchunk;
+                const ExpertDev &ex = fa.experts[E + q];
+                const int row0 = (item - q * nchunk) * 32 + (c2.m % spm) * R;
+                bulk_prefetch_l2((c2.m < spm ? ex.gate.codes : ex.up.codes) + (size_t)row0 * RB, (uint32_t)gu_bytes);
+                c2.next(1 << 30, steps, subs);
+            }
             for (int i = 0; i < S; ++i)
                 bulk_prefetch_l2(fa.experts[E + i].down.codes + (size_t)r0 * RBI, (uint32_t)(nrows * RBI));
+        }
         __syncwarp();
         named_bar(2, DECODE_THREADS);        // routing tables ready (or aborted)
         if (*abort) {
@@ -1135,10 +1207,17 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         // memory
         const uint8_t **ptab = reinterpret_cast<const uint8_t **>(smem + L.eptr);
         for (int a = lane; a < n_active; a += 32) {
-            const ExpertDev ex = fa.experts[lw.active[a]];
-            ptab[3 * a] = ex.gate.codes;
-            ptab[3 * a + 1] = ex.up.codes;
-            ptab[3 * a + 2] = ex.down.codes;
+            const int e = lw.active[a];
+            if (fa.ptr_smem) {
+                ptab[3 * a] = static_cast<const uint8_t *>(eptrs[4 * e]);
+                ptab[3 * a + 1] = static_cast<const uint8_t *>(eptrs[4 * e + 1]);
+                ptab[3 * a + 2] = static_cast<const uint8_t *>(eptrs[4 * e + 2]);
+            } else {
+                const ExpertDev ex = fa.experts[e];
+                ptab[3 * a] = ex.gate.codes;
+                ptab[3 * a + 1] = ex.up.codes;
+                ptab[3 * a + 2] = ex.down.codes;
+            }
         }
         __syncwarp();
         if (lane != 0) return;
@@ -1166,9 +1245,21 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         // No L2 prefetch ahead of the ring: the bulk-copy unit of the SM is
         // what limits the issue rate, and a prefetch costs it as much as the
         // copy itself; ns stages in flight already cover the DRAM latency.
+        long long si = issued;  // ring slots filled so far
         for (int st = issued; st < n_total; ++st) {
-            if (st >= ns && !mbar_wait_sleepy(&bars->empty[rp.slot], rp.phase ^ 1u, fa.err)) {
-                pipe_drain(bars, ns, st, st - ns, fa.err);
+            // a down stage may take two adjacent slots (it starts on an even
+            // slot: every gate/up item is an even number of stages and ns is
+            // even then); both must be free
+            const int span = cur.down ? fa.down_span : 1;
+            RingPos wp = rp;
+            bool free_ok = true;
+            for (int z = 0; z < span && free_ok; ++z) {
+                if (si + z >= ns && !mbar_wait_sleepy(&bars->empty[wp.slot], wp.phase ^ 1u, fa.err))
+                    free_ok = false;
+                wp.next(ns);
+            }
+            if (!free_ok) {
+                pipe_drain(bars, ns, si, si - ns > 0 ? si - ns : 0, fa.err);
                 return;
             }
             uint32_t bytes;
@@ -1176,74 +1267,41 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
             mbar_expect_tx(&bars->full[rp.slot], bytes);
             bulk_g2s_hint(ring + (size_t)rp.slot * PIPE_STAGE_MAX, src, bytes, &bars->full[rp.slot], pol);
             rp.next(ns);
+            for (int z = 1; z < span; ++z) {  // the second slot's phase completes with no data
+                mbar_arrive(&bars->full[rp.slot]);
+                rp.next(ns);
+            }
+            si += span;
             cur.next(my_items, steps, subs);
         }
         return;  // the consumers wait for every copy
     }
 
-    if (warp == PIPE_CONSUMERS + 1) {
-        // ------------------------------ epilogue warp: SwiGLU + Q8_0(h) of
-        // every item, off the consumers' critical path
+    if (warp == PIPE_CONSUMERS + 2) {
+        // ------------------------------ h-fetch warp: the h records of every
+        // active expert, in the down order, into the nh shared slots as soon
+        // as all its gate/up items (any CTA's) are counted -- many experts'
+        // copies in flight at once, and no grid barrier: a CTA starts its
+        // down rows of an expert as soon as that expert's h is complete.
         named_bar(2, DECODE_THREADS);
         bool ok = !*abort;
+        const int nh = fa.nh;
         if (ok) {
             const int n_active = *lw.n_active;
-            const int n_items = n_active * nchunk;
-            int n = 0;
-            for (int item = blockIdx.x; item < n_items && ok; item += G, ++n) {
-                const int buf = n & 1;
-                int a, e, c;
-                item_expert_chunk(item, n_active, a, e, c);
-                if (e < 0) e = lw.active[a];
-                const int p0 = lw.off[a];
-                const int ne = min(lw.off[a + 1] - p0, PIPE_MAX_TOK);
-                const ExpertDev ex = fa.experts[e];
-                const float sg = __ldg(ex.gate.scales + c * 32 + lane);
-                const float su = __ldg(ex.up.scales + c * 32 + lane);
-                if (!mbar_wait_sleepy(&ebars->part_full[buf], (uint32_t)((n >> 1) & 1), fa.err)) {
+            // slots in the x records' space: only once every consumer warp is done with them
+            if (fa.h_alias && !mbar_wait_sleepy(xfree, 0, fa.err)) ok = false;
+            for (int q = 0; ok && q < n_active; ++q) {
+                const int a = down_slot(q, n_active, S), slot = q % nh;
+                if (q >= nh && !mbar_wait_sleepy(&hempty[slot], (uint32_t)((q / nh - 1) & 1), fa.err)) {
                     ok = false;
-                    *abort = 1;
-                    break;
-                }
-                const double *pbuf = part + (size_t)buf * 2 * part_mat;
-                for (int i = 0; i < ne; ++i) {
-                    double ag = 0.0, au = 0.0;
-                    for (int sl = 0; sl < slices; ++sl) {
-                        ag += pbuf[((size_t)lane * slices + sl) * ntok + i];
-                        au += pbuf[part_mat + ((size_t)lane * slices + sl) * ntok + i];
-                    }
-                    const float g = (float)(ag * (double)sg);
-                    const float u = (float)(au * (double)su);
-                    const double gd = (double)g;
-                    const float h = (float)((gd / (1.0 + exp(-gd))) * (double)u);
-                    const int pr = p0 + i;
-                    q8_block_to_record<BITS>(h, c, I, fa.hrec + (size_t)pr * rbI,
-                                             fa.hq + (int64_t)pr * I, fa.hd + (int64_t)pr * (I / COLI_QBLK));
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&ebars->part_free[buf]);
-                    __threadfence();  // the item's h records before its count
-                    atomicAdd(fa.hcnt + a, 1);
-                }
-            }
-        }
-        // then the h records of every active expert, in the down order, into
-        // two shared slots, each once all its gate/up items (any CTA's) are
-        // counted -- this replaces a grid barrier: a CTA starts its down rows
-        // of an expert as soon as that expert's h is complete
-        if (ok && !*abort) {
-            const int n_active = *lw.n_active;
-            for (int q = 0; q < n_active; ++q) {
-                const int a = down_slot(q, n_active, S), slot = q & 1;
-                if (q >= 2 && !mbar_wait_sleepy(&ebars->h_empty[slot], (uint32_t)(((q >> 1) - 1) & 1), fa.err)) {
-                    *abort = 1;
                     break;
                 }
                 int ready = 1;
                 if (lane == 0) {
+                    // relaxed polls with a back-off (no fence per poll), then
+                    // one acquire of the complete count
                     const long long t0 = clock64();
-                    while ((int)ld_acquire_u32(reinterpret_cast<const unsigned *>(fa.hcnt + a)) < nchunk) {
+                    while ((int)ld_relaxed_u32(reinterpret_cast<const unsigned *>(fa.hcnt + a)) < nchunk) {
                         if (*abort) {
                             ready = 0;
                             break;
@@ -1253,20 +1311,81 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
                             ready = 0;
                             break;
                         }
-                        __nanosleep(64);
+                        __nanosleep(200);
                     }
+                    if (ready && (int)ld_acquire_u32(reinterpret_cast<const unsigned *>(fa.hcnt + a)) < nchunk)
+                        ready = 0;  // unreachable: the count never decreases within a launch
                 }
                 ready = __shfl_sync(0xffffffffu, ready, 0);
+                __syncwarp();  // every lane's reads below come after lane 0's acquire
                 if (!ready) {
-                    *abort = 1;
+                    ok = false;
                     break;
                 }
                 const int p0 = lw.off[a], ne = lw.off[a + 1] - p0;
-                const uint4 *src = reinterpret_cast<const uint4 *>(fa.hrec + (size_t)p0 * rbI);
-                uint4 *dst = reinterpret_cast<uint4 *>(acts + (size_t)slot * T * rbI);
-                for (int i = lane; i < ne * rbI / 16; i += 32) dst[i] = __ldcg(src + i);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&ebars->h_full[slot]);
+                const uint8_t *src = fa.hrec + (size_t)p0 * rbI;
+                uint8_t *dst = hslots + (size_t)slot * T * rbI;
+                for (int i = lane; i < ne * rbI / 16; i += 32) cp_async16(dst + 16 * i, src + 16 * i);
+                cp_async_arrive_noinc(&hfull[slot]);  // each lane: once its copies land
+            }
+        }
+        if (!ok) *abort = 1;
+        cp_async_wait_all();  // no copy lands in shared memory after this warp leaves
+        return;
+    }
+
+    if (warp == PIPE_CONSUMERS + 1) {
+        // ------------------------------ epilogue warp.  While routing runs:
+        // every expert's code pointers into shared memory (ptr_smem).  P3:
+        // SwiGLU + Q8_0(h) of every item, off the consumers' critical path;
+        // each item's count is released once its h records are written.
+        if (fa.ptr_smem) {
+            for (int e = lane; e < E + S; e += 32) {
+                const ExpertDev &ex = fa.experts[e];
+                eptrs[4 * e] = ex.gate.codes;
+                eptrs[4 * e + 1] = ex.up.codes;
+                eptrs[4 * e + 2] = ex.down.codes;
+                eptrs[4 * e + 3] = ex.down.scales;
+            }
+        }
+        named_bar(2, DECODE_THREADS);
+        if (*abort) return;
+        const int n_active = *lw.n_active;
+        const int n_items = n_active * nchunk;
+        int n = 0;
+        for (int item = blockIdx.x; item < n_items; item += G, ++n) {
+            const int buf = n & 1;
+            int a, e, c;
+            item_expert_chunk(item, n_active, a, e, c);
+            if (e < 0) e = lw.active[a];
+            const int p0 = lw.off[a];
+            const int ne = min(lw.off[a + 1] - p0, PIPE_MAX_TOK);
+            const ExpertDev ex = fa.experts[e];
+            const float sg = __ldg(ex.gate.scales + c * 32 + lane);
+            const float su = __ldg(ex.up.scales + c * 32 + lane);
+            if (!mbar_wait_sleepy(&ebars->part_full[buf], (uint32_t)((n >> 1) & 1), fa.err)) {
+                *abort = 1;
+                break;
+            }
+            const double *pbuf = part + (size_t)buf * 2 * part_mat;
+            for (int i = 0; i < ne; ++i) {
+                double ag = 0.0, au = 0.0;
+                for (int sl = 0; sl < slices; ++sl) {
+                    ag += pbuf[((size_t)lane * slices + sl) * ntok + i];
+                    au += pbuf[part_mat + ((size_t)lane * slices + sl) * ntok + i];
+                }
+                const float g = (float)(ag * (double)sg);
+                const float u = (float)(au * (double)su);
+                const double gd = (double)g;
+                const float h = (float)((gd / (1.0 + exp(-gd))) * (double)u);
+                const int pr = p0 + i;
+                q8_block_to_record<BITS>(h, c, I, fa.hrec + (size_t)pr * rbI,
+                                         fa.hq + (int64_t)pr * I, fa.hd + (int64_t)pr * (I / COLI_QBLK));
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&ebars->part_free[buf]);
+                red_release_add(fa.hcnt + a, 1);  // the item's h records before its count
             }
         }
         return;
@@ -1275,9 +1394,9 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
     // ---------------------------------- consumers
     // P1: logits of experts b, b + G, ... (two per pass, loads issued four
     // iterations at a time) and a share of Q8_0(x).  Every consumer thread
-    // first requests its first router-weight lines into L2 and then, without
-    // condition, releases the producer (barrier 4), so those requests enter
-    // the memory queues ahead of the shared-expert bulk copies.
+    // first requests its first router-weight lines into L2; the producer's
+    // shared-expert bulk copies wait (barrier 4) until the selection's scores
+    // are loaded, so the latency-bound routing steps do not queue behind them.
     if ((int)blockIdx.x < E) {
         const int e1 = (int)blockIdx.x + G;
         for (int i = tid; i < H / 4 && i < 4 * 256; i += 256) {
@@ -1285,8 +1404,6 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
             if (e1 < E) asm volatile("prefetch.global.L2 [%0];" ::"l"(fa.Wr + (int64_t)e1 * H + 4 * i));
         }
     }
-    __syncwarp();
-    asm volatile("bar.arrive 4, %0;" ::"r"(32 * (PIPE_CONSUMERS + 1)) : "memory");
     for (int e0 = blockIdx.x; e0 < E; e0 += 2 * G) {
         const int e1 = e0 + G;
         const bool two = e1 < E;
@@ -1368,15 +1485,19 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
     named_bar(1, 256);
     if (!flags[0]) {
         *abort = 1;
+        __syncwarp();  // the producer still waits at barrier 4
+        asm volatile("bar.arrive 4, %0;" ::"r"(32 * (PIPE_CONSUMERS + 1)) : "memory");
     } else {
         // P2: x records (async, overlapping the selection), selection, union
         for (int i = tid; i < T * rbH / 16; i += 256) cp_async16(acts + 16 * i, fa.xrec + 16 * i);
         const bool pub = blockIdx.x == 0;
         for (int t = 0; t < T; ++t) {
             sm.w_smem = w_s + t * k;
+            // the first token's scores loaded: release the producer (barrier 4)
             cta_select_token<SyncConsumers>(fa.ws.c + (int64_t)t * E, fa.ws.s + (int64_t)t * E, E,
                                             fa.G, fa.gk, k, fa.rsf, sm, pub ? fa.ws.idx + t * k : nullptr,
-                                            pub ? fa.ws.w + t * k : nullptr, idx_s + t * k);
+                                            pub ? fa.ws.w + t * k : nullptr, idx_s + t * k, 4,
+                                            t == 0 ? 32 * (PIPE_CONSUMERS + 1) : 0);
         }
         if (MAXT == 1) {
             if (warp == 0) warp_union_one(lw, E, S, k, idx_s);
@@ -1401,10 +1522,25 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
     named_bar(2, DECODE_THREADS);        // tables ready: release producer and epilogue warp
     if (consumers_aborted(abort, flags + 1)) return;
 
+    // down-row scales of this CTA's rows for every active expert (they need
+    // no h): 4-byte async copies, landing while the gate/up items run
+    const int n_active = *lw.n_active;
+    {
+        const int ds = fa.rows_cap + 4;
+        for (int i = tid; i < n_active * nrows; i += 256) {
+            const int a = i / nrows, r = i % nrows;
+            const int e = lw.active[a];
+            const float *dsc = fa.ptr_smem ? static_cast<const float *>(eptrs[4 * e + 3])
+                                           : fa.experts[e].down.scales;
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dscale + a * ds + r)),
+                         "l"(dsc + r0 + r)
+                         : "memory");
+        }
+    }
+
     // P3: gate/up items; partials go to the epilogue warp through part_full /
     // part_free (two buffers)
     const FastGeo fgeo(geo, V);
-    const int n_active = *lw.n_active;
     const int n_items = n_active * nchunk;
     RingPos rp;
     bool ok = true;
@@ -1464,24 +1600,14 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         __syncwarp();
         if (lane == 0) mbar_arrive(&ebars->part_full[buf]);
     }
-    // down-row scales of this CTA's rows for every active expert (they need
-    // no h): 4-byte async copies
-    if (!*abort) {
-        const int ds = fa.rows_cap + 4;
-        for (int i = tid; i < n_active * nrows; i += 256) {
-            const int a = i / nrows, r = i % nrows;
-            const float *src = fa.experts[lw.active[a]].down.scales + r0 + r;
-            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dscale + a * ds + r)),
-                         "l"(src)
-                         : "memory");
-        }
-    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(xfree);  // no x record is read after this
     cp_async_wait_all();
     if (consumers_aborted(abort, flags + 1)) return;
     // P4: down rows of every active expert as its h arrives, then the combine
     const int vpl = (VI % 32 == 0) ? VI / 32 : 0;
     DownLoop dl{lw.off, n_active, S, T, subs, ns, fa.down_rows, fa.rows_cap, r0, nrows, RBI, VI, I, rbI,
-                ring, dscale, acts, ebuf, bars, ebars, abort, fa.err};
+                fa.down_span, ring, dscale, hslots, fa.nh, hfull, hempty, ebuf, bars, abort, fa.err};
     switch (vpl) {
         case 1: ok = down_loop<BITS, 1, MAXT>(dl, rp) && ok; break;
         case 2: ok = down_loop<BITS, 2, MAXT>(dl, rp) && ok; break;

@@ -166,24 +166,28 @@ __device__ __forceinline__ int block_exscan256(int v, int *tmp /*[8]*/, int &tot
 // Selection of one token by a whole CTA (256 threads), rank based, no serial
 // scans:  in-group ranks give each group's two best c (its score); group
 // ranks keep the topk_group best groups; the top_k of the kept experts are
-// among the experts ranked < top_k inside their own kept group, and their
+// among the min(top_k, E/G) experts ranked first inside their own kept group,
+// which are laid out densely (kept-group position x in-group rank), and their
 // ranks among those candidates give idx sorted by descending c.  Every
-// comparison breaks ties toward the lower index.
+// comparison breaks ties toward the lower index.  Each step is a loop of
+// independent shared-memory reads, so it runs at the load issue rate rather
+// than at the latency of a dependent chain.
 struct SelectSmem {
     double *c;      // [E]
     double *s;      // [E]
+    double *candc;  // [E] choice scores of the candidates, in candidate order
     int *grank;     // [E] rank inside its group
     double *top1;   // [G]
-    double *top2;   // [G]
-    int *keep;      // [G]
-    int *cand;      // [E]
+    double *top2;   // [G] second best, then the group score
+    int *keep;      // [G] 1 if kept, then its position among the kept groups (-1: dropped)
+    int *cand;      // [E] expert of each candidate
     int *ncand;     // [1]
     int *sel;       // [32]
     float *w_smem;  // optional [k] copy of the weights (set by the caller)
 };
 
 __host__ __device__ inline size_t select_smem_bytes(int E, int G) {
-    return (size_t)E * 16 + (size_t)G * 16 + (size_t)E * 8 + (size_t)G * 4 + 4 + 32 * 4 + 64;
+    return (size_t)E * 24 + (size_t)G * 16 + (size_t)E * 8 + (size_t)G * 4 + 4 + 32 * 4 + 64;
 }
 
 __device__ inline SelectSmem carve_select(void *base, int E, int G) {
@@ -191,6 +195,7 @@ __device__ inline SelectSmem carve_select(void *base, int E, int G) {
     char *p = (char *)base;
     m.c = (double *)p;           p += (size_t)E * 8;
     m.s = (double *)p;           p += (size_t)E * 8;
+    m.candc = (double *)p;       p += (size_t)E * 8;
     m.top1 = (double *)p;        p += (size_t)G * 8;
     m.top2 = (double *)p;        p += (size_t)G * 8;
     m.grank = (int *)p;          p += (size_t)E * 4;
@@ -202,76 +207,214 @@ __device__ inline SelectSmem carve_select(void *base, int E, int G) {
     return m;
 }
 
+// Warp-level selection for the common shape: every group fits one warp
+// (E/G <= 32), at most 8 groups, and the kept groups' candidates fit one warp
+// (topk_group * min(top_k, E/G) <= 32).  Warp g holds group g, one expert per
+// lane; ranks come from branch-free shuffle comparisons (ties: lower index),
+// and only three CTA barriers are taken.  Same results as the general path.
+__host__ __device__ inline bool select_warp_shape(int E, int G, int gk, int k) {
+    const int per = E / G, kk = k < per ? k : per;
+    return per <= 32 && G <= 8 && gk * kk <= 32 && k <= 32;
+}
+
+template <typename Sync>
+__device__ void cta_select_token_warps(const double *c_row, const double *s_row, int E, int G,
+                                       int gk, int k, float rsf, const SelectSmem &sm,
+                                       int32_t *idx_out, float *w_out, int *idx_smem,
+                                       int arrive_bar, int arrive_count) {
+    const unsigned FULL = 0xffffffffu;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int per = E / G, kk = k < per ? k : per;
+    const int e = warp * per + lane;
+    const bool mine = warp < G && lane < per;
+    double v = 0.0, sv = 0.0;
+    if (mine) {
+        v = __ldcg(c_row + e);
+        sv = __ldcg(s_row + e);
+    }
+    int r = 0;
+    if (warp < G) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const double u = __shfl_sync(FULL, v, j);
+            r += (int)(j < per) & ((int)(u > v) | ((int)(u == v) & (int)(j < lane)));
+        }
+        // the group's score: its best c plus its second best
+        const unsigned m0 = __ballot_sync(FULL, mine && r == 0);
+        const unsigned m1 = __ballot_sync(FULL, mine && r == 1);
+        const double t1 = __shfl_sync(FULL, v, __ffs(m0) - 1);
+        const double t2 = __shfl_sync(FULL, v, m1 ? __ffs(m1) - 1 : 0);
+        if (lane == 0) sm.top2[warp] = t1 + (per > 1 ? t2 : 0.0);
+    }
+    if (arrive_count > 0) {  // this thread's scores (r used them) and async copies have landed
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncwarp();
+        asm volatile("bar.arrive %0, %1;" ::"r"(arrive_bar), "r"(arrive_count) : "memory");
+    }
+    Sync::sync();
+    // every warp: the ranks of the G group scores, the kept groups
+    const double gsv = lane < G ? sm.top2[lane] : 0.0;
+    int grk = 0;
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+        const double u = __shfl_sync(FULL, gsv, h);
+        grk += (int)(h < G) & ((int)(u > gsv) | ((int)(u == gsv) & (int)(h < lane)));
+    }
+    const unsigned kept = __ballot_sync(FULL, lane < G && grk < gk);
+    if (warp < G && ((kept >> warp) & 1u) && mine && r < kk) {
+        const int pos = __popc(kept & ((1u << warp) - 1u)) * kk + r;
+        sm.cand[pos] = e;
+        sm.candc[pos] = v;
+        sm.s[pos] = sv;
+    }
+    Sync::sync();
+    if (warp == 0) {
+        const int n = gk * kk;
+        const bool has = lane < n;
+        const double cv = has ? sm.candc[lane] : 0.0;
+        const int ce = has ? sm.cand[lane] : 0;
+        const double cs = has ? sm.s[lane] : 0.0;
+        int rank = 0;
+#pragma unroll 8
+        for (int j = 0; j < n; ++j) {  // broadcast reads of every candidate
+            const double u = sm.candc[j];
+            const int f = sm.cand[j];
+            rank += (int)(u > cv) | ((int)(u == cv) & (int)(f < ce));
+        }
+        // slot j is the candidate of rank j; the weights renormalise s over
+        // the slots in slot order, times rsf
+        __syncwarp();
+        if (has && rank < k) {
+            sm.sel[rank] = ce;
+            sm.c[rank] = cs;
+        }
+        __syncwarp();
+        double ssum = 0.0;
+#pragma unroll 8
+        for (int j = 0; j < k; ++j) ssum += sm.c[j];
+        if (lane < k) {
+            const int ej = sm.sel[lane];
+            const float wj = (float)((sm.c[lane] / ssum) * (double)rsf);
+            if (idx_out) idx_out[lane] = ej;
+            if (w_out) w_out[lane] = wj;
+            if (idx_smem) idx_smem[lane] = ej;
+            if (sm.w_smem) sm.w_smem[lane] = wj;
+        }
+    }
+    Sync::sync();
+}
+
+// arrive_bar / arrive_count: if arrive_count > 0, every calling thread
+// arrives (bar.arrive) on that named barrier as soon as the token's scores
+// and the thread's earlier cp.async copies have landed -- a hook for a warp
+// that must not start memory traffic before those loads are done.
 template <typename Sync = SyncAll>
 __device__ void cta_select_token(const double *c_row, const double *s_row, int E, int G, int gk,
                                  int k, float rsf, const SelectSmem &sm, int32_t *idx_out,
-                                 float *w_out, int *idx_smem = nullptr) {
+                                 float *w_out, int *idx_smem = nullptr, int arrive_bar = 0,
+                                 int arrive_count = 0) {
+    if (select_warp_shape(E, G, gk, k)) {
+        cta_select_token_warps<Sync>(c_row, s_row, E, G, gk, k, rsf, sm, idx_out, w_out, idx_smem,
+                                     arrive_bar, arrive_count);
+        return;
+    }
     const int tid = threadIdx.x, nthr = 256;
     const int per = E / G;
+    const int kk = k < per ? k : per;  // candidates one kept group can contribute
     for (int e = tid; e < E; e += nthr) {
         sm.c[e] = __ldcg(c_row + e);
         sm.s[e] = __ldcg(s_row + e);
     }
-    if (tid == 0) *sm.ncand = 0;
     Sync::sync();
+    if (arrive_count > 0) {  // this thread's scores and async copies have landed
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncwarp();
+        asm volatile("bar.arrive %0, %1;" ::"r"(arrive_bar), "r"(arrive_count) : "memory");
+    }
     for (int e = tid; e < E; e += nthr) {
-        const int g = e / per;
+        const int g = e / per, g0 = g * per;
         const double v = sm.c[e];
         int r = 0;
+#pragma unroll 8
         for (int i = 0; i < per; ++i) {
-            const int f = g * per + i;
-            const double u = sm.c[f];
-            r += (u > v) || (u == v && f < e);
+            const double u = sm.c[g0 + i];
+            r += (int)(u > v) | ((int)(u == v) & (int)(g0 + i < e));
         }
         sm.grank[e] = r;
         if (r == 0) sm.top1[g] = v;
         if (r == 1) sm.top2[g] = v;
     }
     Sync::sync();
-    for (int g = tid; g < G; g += nthr) {
-        const double v = sm.top1[g] + (per > 1 ? sm.top2[g] : 0.0);
-        sm.top2[g] = v;  // reuse: group score
-    }
+    for (int g = tid; g < G; g += nthr) sm.top2[g] = sm.top1[g] + (per > 1 ? sm.top2[g] : 0.0);
     Sync::sync();
     for (int g = tid; g < G; g += nthr) {
         const double v = sm.top2[g];
         int r = 0;
+#pragma unroll 8
         for (int h = 0; h < G; ++h) {
             const double u = sm.top2[h];
-            r += (u > v) || (u == v && h < g);
+            r += (int)(u > v) | ((int)(u == v) & (int)(h < g));
         }
         sm.keep[g] = r < gk;
     }
     Sync::sync();
-    for (int e = tid; e < E; e += nthr)
-        if (sm.keep[e / per] && sm.grank[e] < k) sm.cand[atomicAdd(sm.ncand, 1)] = e;
+    // position of each kept group among the kept groups (index order)
+    if (G <= nthr) {
+        int kpos = -1;
+        if (tid < G) {
+            int before = 0;
+#pragma unroll 8
+            for (int h = 0; h < tid; ++h) before += sm.keep[h];
+            kpos = sm.keep[tid] ? before : -1;
+        }
+        Sync::sync();
+        if (tid < G) sm.keep[tid] = kpos;
+    } else if (tid == 0) {
+        int n = 0;
+        for (int g = 0; g < G; ++g) sm.keep[g] = sm.keep[g] ? n++ : -1;
+    }
     Sync::sync();
-    const int n = *sm.ncand;
+    for (int e = tid; e < E; e += nthr) {
+        const int pos = sm.keep[e / per];
+        const int r = sm.grank[e];
+        if (pos >= 0 && r < kk) {
+            sm.cand[pos * kk + r] = e;
+            sm.candc[pos * kk + r] = sm.c[e];
+        }
+    }
+    Sync::sync();
+    const int n = gk * kk;
     for (int i = tid; i < n; i += nthr) {
+        const double v = sm.candc[i];
         const int e = sm.cand[i];
-        const double v = sm.c[e];
         int r = 0;
+#pragma unroll 8
         for (int j = 0; j < n; ++j) {
+            const double u = sm.candc[j];
             const int f = sm.cand[j];
-            const double u = sm.c[f];
-            r += (u > v) || (u == v && f < e);
+            r += (int)(u > v) | ((int)(u == v) & (int)(f < e));
         }
         if (r < k) sm.sel[r] = e;
     }
     Sync::sync();
-    if (tid == 0) {
-        double ssum = 0.0;  // slot order, as the weights' definition sums
-        for (int j = 0; j < k; ++j) ssum += sm.s[sm.sel[j]];
-        sm.c[0] = ssum;     // c is no longer needed
-    }
-    Sync::sync();
-    if (tid < k) {
-        const int e = sm.sel[tid];
-        const float wj = (float)((sm.s[e] / sm.c[0]) * (double)rsf);
-        if (idx_out) idx_out[tid] = e;
-        if (w_out) w_out[tid] = wj;
-        if (idx_smem) idx_smem[tid] = e;
-        if (sm.w_smem) sm.w_smem[tid] = wj;
+    if (tid < 32) {
+        // weights: s of the selection renormalised (sum in slot order) x rsf
+        const int lane = tid;
+        const int e = lane < k ? sm.sel[lane] : 0;
+        const double sj = lane < k ? sm.s[e] : 0.0;
+        double ssum = 0.0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const double v = __shfl_sync(0xffffffffu, sj, j);
+            if (j < k) ssum += v;
+        }
+        if (lane < k) {
+            const float wj = (float)((sj / ssum) * (double)rsf);
+            if (idx_out) idx_out[lane] = e;
+            if (w_out) w_out[lane] = wj;
+            if (idx_smem) idx_smem[lane] = e;
+            if (sm.w_smem) sm.w_smem[lane] = wj;
+        }
     }
     Sync::sync();
 }

@@ -217,11 +217,23 @@ def test_glm52_verify_t4_shares_experts(glm52_layer):
     assert len(a & b) >= 1, "tokens 0 and 1 share no expert"
 
 
-def test_glm52_prefill_t2048_sampled(glm52_layer):
+def _compare_on_tensor_cores(gl, x):
+    """compare_forward on every token, asserting that the forward ran the
+    tcgen05 grouped GEMMs (not the CUDA-core grouped kernels)."""
+    gl.handle.profile(True)
+    compare_forward(gl, x)
+    names = gl.handle.profile_read()
+    gl.handle.profile(False)
+    assert "gateup_tc" in names and "down_tc" in names, sorted(names)
+
+
+def test_glm52_prefill_t2048_every_token(glm52_layer):
+    """Batch-union prefill of 2048 tokens: every token's routing, Q8_0(h)
+    codes of all 9 slots and output row against the oracle, on the tensor-core
+    path (every one of the 257 experts is active)."""
     cfg = synth.workload("glm52_prefill_int4_t2048")
     x = synth.tokens(cfg, device=DEV)
-    sample = [0, 1, 2, 511, 1024, 1500, 2046, 2047]
-    compare_forward(glm52_layer, x, tokens=sample)
+    _compare_on_tensor_cores(glm52_layer, x)
 
 
 @pytest.mark.parametrize("bits", [8, 2])
@@ -230,7 +242,9 @@ def test_glm52_sweep_formats(bits, T):
     cfg = synth.workload("glm52_sweep", bits=bits)
     gl = GpuLayer(cfg, max_tokens=T)
     x = synth.tokens(cfg, T=T, device=DEV)
-    sample = list(range(T)) if T <= 4 else [0, 7, 255, 511]
-    compare_forward(gl, x, tokens=sample)
+    if T > 8:
+        _compare_on_tensor_cores(gl, x)
+    else:
+        compare_forward(gl, x)
     gl.close()
     torch.cuda.empty_cache()
