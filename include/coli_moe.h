@@ -235,6 +235,17 @@ coli_status coli_router_static(const coli_moe_config *cfg, const float *router_w
                                const float *bias, const float *x, int T, int32_t *idx, float *w,
                                coli_stream_t stream);
 
+/* Test hook for the bounded waits of the layer's own kernels (no counterpart
+ * on the pages).  Sets how many SM cycles a wait on another part of a kernel
+ * may last before that kernel gives up (records COLI_ETIMEOUT in the handle's
+ * error word, leaves without finishing the call, and the call's outputs are
+ * undefined); cycles <= 0 restores the default of about one second.  Waits for
+ * work already issued (bulk copies, tensor-core MMAs) keep the default, so a
+ * kernel that gives up still leaves no copy in flight and no tensor memory
+ * held.  Applies to later calls on this handle; returns once the new limit is
+ * in place. */
+coli_status coli_dbg_set_wait_limit(coli_moe *m, long long cycles, coli_stream_t stream);
+
 /* Test hook for the bounded waits (no counterpart on the pages): one thread
  * waits on an mbarrier that nothing ever arrives at, through the same bounded
  * wait the pipelined kernels use.  The wait gives up after about one second

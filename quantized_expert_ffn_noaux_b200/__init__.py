@@ -80,6 +80,7 @@ def lib():
         "coli_dbg_block_sums": ([vp, ci, i64, i64, vp, ci, vp, vp], ci),
         "coli_dbg_last_forward": ([vp, ci, vp, vp, vp, vp, vp], ci),
         "coli_dbg_wait_probe": ([vp, vp], ci),
+        "coli_dbg_set_wait_limit": ([vp, ctypes.c_longlong, vp], ci),
         "coli_moe_device_status": ([vp, vp], ci),
         "coli_router_static": ([vp, vp, vp, vp, ci, vp, vp, vp], ci),
     }
@@ -259,6 +260,10 @@ class MoELayer:
 
     def dbg_wait_probe(self, stream=None):
         _check(lib().coli_dbg_wait_probe(self._h, _stream(stream)))
+
+    def dbg_set_wait_limit(self, cycles, stream=None):
+        """Cycles a kernel wait on progress may last (<= 0: the default)."""
+        _check(lib().coli_dbg_set_wait_limit(self._h, int(cycles), _stream(stream)))
 
     def dbg_last_forward(self, T, stream=None):
         c = self.cfg

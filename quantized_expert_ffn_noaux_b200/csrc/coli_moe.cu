@@ -106,7 +106,8 @@ struct coli_moe {
     uint8_t *xrec = nullptr, *hrec = nullptr;
     int *err = nullptr;
     unsigned long long *gbar = nullptr;
-    int *hcnt = nullptr;  // per active expert: gate/up items done (decode kernel)  // grid-barrier arrival counter of the decode kernel
+    int *hcnt = nullptr;  // per active expert: gate/up items done (decode kernel)
+    long long *wait_limit = nullptr;  // SM cycles a kernel's wait on progress may last
     int last_T = 0;
     std::map<const void *, int> occ_cache;  // kernel -> CTAs per SM (attributes already set)
     // profiling
@@ -130,7 +131,7 @@ struct WsOffsets {
     size_t s, c, idx, w, bitmap, prefix, counter, n_active, active, off, act_of, pair_tok,
         pair_slot, tok_pair, xq, xd, hq, hd, e_pairs, xg, xdg, maps, corr_x, corr_h, x_in, y_out, experts,
         xrec, hrec,
-        err, gbar, hcnt;
+        err, gbar, hcnt, wait_limit;
     size_t total;
 };
 
@@ -199,6 +200,7 @@ WsOffsets layout_of(const coli_moe_config &c) {
     o.err = L.add(4);
     o.gbar = L.add(8);
     o.hcnt = L.add((E + S) * 4);
+    o.wait_limit = L.add(8);
     o.total = L.total;
     return o;
 }
@@ -562,6 +564,7 @@ coli_status launch_small_path(coli_moe *m, const float *x, int T, float *out, cu
     fa.hd = m->hd;
     fa.out = out;
     fa.err = m->err;
+    fa.wait_limit = m->wait_limit;
     fa.gbar = m->gbar;
     fa.hcnt = m->hcnt;
     fa.ns = p.ns;
@@ -663,6 +666,7 @@ coli_status launch_grouped_tc(coli_moe *m, int T, int down, cudaStream_t s) {
     ta.hd = m->hd;
     ta.e_pairs = m->e_pairs;
     ta.err = m->err;
+    ta.wait_limit = m->wait_limit;
     Launch L(m, s, down ? "down_tc" : "gateup_tc");
     kern<<<m->nsm, TC_THREADS, smem, s>>>(ta);
     return L.done();
@@ -946,9 +950,14 @@ coli_status coli_moe_create(const coli_moe_config *cfg, const float *router_w, c
     m->err = (int *)(b + o.err);
     m->gbar = (unsigned long long *)(b + o.gbar);
     m->hcnt = (int *)(b + o.hcnt);
+    m->wait_limit = (long long *)(b + o.wait_limit);
     e = cudaMemset(m->ws_base, 0, o.total);
     if (e == cudaSuccess)
         e = cudaMemcpy(m->experts_dev, host.data(), sizeof(ExpertDev) * n, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) {
+        const long long lim = WAIT_LIMIT_CYCLES;
+        e = cudaMemcpy(m->wait_limit, &lim, sizeof lim, cudaMemcpyHostToDevice);
+    }
     if (e == cudaSuccess && m->maps_dev) {
         // the tensor-core path's maps; any shape or alignment the copy engine
         // refuses leaves that path off (the CUDA-core grouped kernels run)
@@ -1147,6 +1156,19 @@ coli_status coli_dbg_wait_probe(coli_moe *m, coli_stream_t stream) {
     Launch L(nullptr, s, "dbg_wait_probe");
     k_dbg_wait_probe<<<1, 32, 0, s>>>(m->err);
     return L.done();
+}
+
+coli_status coli_dbg_set_wait_limit(coli_moe *m, long long cycles, coli_stream_t stream) {
+    g_last_error.clear();
+    coli_status st = check_handle(m);
+    if (st != COLI_OK) return st;
+    const long long lim = cycles > 0 && cycles < WAIT_LIMIT_CYCLES ? cycles : WAIT_LIMIT_CYCLES;
+    cudaStream_t s = (cudaStream_t)stream;
+    // pageable source: the copy has completed when the call returns
+    COLI_CUDA(cudaMemcpyAsync(m->wait_limit, &lim, sizeof lim, cudaMemcpyHostToDevice, s),
+              "wait limit copy");
+    COLI_CUDA(cudaStreamSynchronize(s), "wait limit copy");
+    return COLI_OK;
 }
 
 coli_status coli_dbg_block_sums(const void *codes, int wfmt, int64_t rows, int64_t K,

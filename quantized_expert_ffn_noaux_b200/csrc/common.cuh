@@ -294,11 +294,12 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parit
         : "memory");
     return ok != 0;
 }
-__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t *bar, uint32_t parity, int *err) {
+__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t *bar, uint32_t parity, int *err,
+                                                 long long lim = WAIT_LIMIT_CYCLES) {
     if (mbar_try_wait_hint(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait_hint(bar, parity)) {
-        if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+        if (clock64() - t0 > lim) {
             if (err) atomicExch(err, ERR_TIMEOUT);
             return false;
         }
@@ -308,12 +309,15 @@ __device__ __forceinline__ bool mbar_wait_sleepy(uint64_t *bar, uint32_t parity,
 }
 
 // Bounded wait for the phase with the given parity; false (and the error
-// word set) if it did not complete within WAIT_LIMIT_CYCLES.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err) {
+// word set) if it did not complete within `lim` SM cycles.  Waits for work
+// that is sure to finish (copies or MMAs already issued) keep the default
+// limit; waits on progress elsewhere may take a shorter per-handle limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err,
+                                          long long lim = WAIT_LIMIT_CYCLES) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+        if (clock64() - t0 > lim) {
             if (err) atomicExch(err, ERR_TIMEOUT);
             return false;
         }

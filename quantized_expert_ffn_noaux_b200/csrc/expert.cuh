@@ -613,6 +613,7 @@ struct RingView {
     int *err;
     volatile int *abort;
     int span = 1;
+    long long lim = WAIT_LIMIT_CYCLES;  // limit of the stage waits
 };
 
 // Consumer side of releasing one (possibly two-slot) stage: every lane has
@@ -643,7 +644,7 @@ __device__ __forceinline__ bool gateup_item_fast(const RingView &rv, RingPos &rp
         double acc[U];
 #pragma unroll
         for (int st = 0; st < SPM; ++st) {
-            if (!mbar_wait(&rv.bars->full[rp.slot], rp.phase, rv.err)) {
+            if (!mbar_wait(&rv.bars->full[rp.slot], rp.phase, rv.err, rv.lim)) {
                 *rv.abort = 1;
                 return false;
             }
@@ -694,7 +695,8 @@ __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned *p) {
 // there (one atomic and, usually, one acquire load per CTA; no reset).
 // Bounded: false (and COLI_ETIMEOUT in *err) if the others did not arrive
 // within WAIT_LIMIT_CYCLES.
-__device__ inline bool grid_barrier(unsigned long long *count, unsigned nblocks, int *err) {
+__device__ inline bool grid_barrier(unsigned long long *count, unsigned nblocks, int *err,
+                                    long long lim) {
     unsigned long long v;
     asm volatile("atom.add.acq_rel.gpu.u64 %0, [%1], 1;" : "=l"(v) : "l"(count) : "memory");
     const unsigned long long target = (v / nblocks + 1) * nblocks;
@@ -703,7 +705,7 @@ __device__ inline bool grid_barrier(unsigned long long *count, unsigned nblocks,
         unsigned long long now;
         asm volatile("ld.acquire.gpu.u64 %0, [%1];" : "=l"(now) : "l"(count) : "memory");
         if (now >= target) return true;
-        if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+        if (clock64() - t0 > lim) {
             atomicExch(err, ERR_TIMEOUT);
             return false;
         }
@@ -782,7 +784,7 @@ __device__ __forceinline__ bool down_expert_deferred(const RingView &rv, RingPos
     for (int i = N; i < U; ++i) acc[i] = 0.0;
 #pragma unroll
     for (int sb = 0; sb < SUBS; ++sb) {
-        if (!mbar_wait(&rv.bars->full[rp.slot], rp.phase, rv.err)) {
+        if (!mbar_wait(&rv.bars->full[rp.slot], rp.phase, rv.err, rv.lim)) {
             *rv.abort = 1;
             return false;
         }
@@ -859,6 +861,7 @@ struct DecodeArgs {
     int nh;             // shared slots for the h records of active experts (<= DECODE_MAX_HSLOTS)
     int h_alias;        // 1: the slots reuse the x records' space, so they fill only after P3
     int ptr_smem;       // 1: every expert's code pointers are staged in shared memory in P1
+    const long long *wait_limit;  // SM cycles a wait on progress may last (drains keep the default)
 };
 
 constexpr int DECODE_MAX_HSLOTS = 16;
@@ -941,6 +944,7 @@ struct EpiBars {
 struct DownLoop {
     const int *off;
     int n_active, S, T, subs, ns, down_rows, rows_cap, r0, nrows, RBI, VI, I, rbI, span;
+    long long lim;
     const uint8_t *ring;
     const float *dscale;
     const uint8_t *hslots;   // nh slots of T h records each, filled by the epilogue warp
@@ -970,7 +974,7 @@ __device__ __forceinline__ bool down_loop(const DownLoop &d, RingPos &rp) {
         // items (any CTA's) are written
         const int hs = q % d.nh;
         const uint8_t *recs = d.hslots + (size_t)hs * d.T * d.rbI;
-        if (!mbar_wait(&d.hfull[hs], (uint32_t)((q / d.nh) & 1), d.err)) {
+        if (!mbar_wait(&d.hfull[hs], (uint32_t)((q / d.nh) & 1), d.err, d.lim)) {
             *d.abort = 1;
             return false;
         }
@@ -982,7 +986,7 @@ __device__ __forceinline__ bool down_loop(const DownLoop &d, RingPos &rp) {
                 act.load(recs, d.I, d.VI, 0);
                 // whole expert at once where the stage geometry allows
                 const float *sc_a = d.dscale + a * (d.rows_cap + 4);
-                const RingView rv{d.ring, d.bars, d.ns, d.err, d.abort, d.span};
+                const RingView rv{d.ring, d.bars, d.ns, d.err, d.abort, d.span, d.lim};
                 if (d.down_rows == 8 * rpw) {
 #define COLI_DEFER(R, SB) done = down_expert_deferred<BITS, VPL, R, SB>(rv, rp, d.RBI, d.nrows, sc_a, act, p0, d.ebuf, d.rows_cap)
                     if (rpw == 6 && d.subs == 1) COLI_DEFER(6, 1);
@@ -1003,7 +1007,7 @@ __device__ __forceinline__ bool down_loop(const DownLoop &d, RingPos &rp) {
             }
         }
         for (int sb = 0; done != 1 && sb < d.subs; ++sb) {
-            if (!mbar_wait(&d.bars->full[rp.slot], rp.phase, d.err)) {
+            if (!mbar_wait(&d.bars->full[rp.slot], rp.phase, d.err, d.lim)) {
                 *d.abort = 1;
                 expert_ok = false;
                 break;
@@ -1086,6 +1090,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
     const int R = geo.R, slices = geo.slices, spm = 32 / R, steps = 2 * spm;
     const int nchunk = I / 32, rbH = rec_bytes(H), rbI = rec_bytes(I), nbH = H / COLI_QBLK;
     const int ns = fa.ns, G = gridDim.x;
+    const long long lim = *fa.wait_limit;
     const DecodeSmem L = decode_smem(T, H, I, E, S, fa.G, k, fa.pmax, slices, fa.rows_cap, ns,
                                      fa.nh, fa.h_alias, fa.ptr_smem);
     uint8_t *ring = smem + L.ring;
@@ -1254,7 +1259,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
             RingPos wp = rp;
             bool free_ok = true;
             for (int z = 0; z < span && free_ok; ++z) {
-                if (si + z >= ns && !mbar_wait_sleepy(&bars->empty[wp.slot], wp.phase ^ 1u, fa.err))
+                if (si + z >= ns && !mbar_wait_sleepy(&bars->empty[wp.slot], wp.phase ^ 1u, fa.err, lim))
                     free_ok = false;
                 wp.next(ns);
             }
@@ -1289,10 +1294,10 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         if (ok) {
             const int n_active = *lw.n_active;
             // slots in the x records' space: only once every consumer warp is done with them
-            if (fa.h_alias && !mbar_wait_sleepy(xfree, 0, fa.err)) ok = false;
+            if (fa.h_alias && !mbar_wait_sleepy(xfree, 0, fa.err, lim)) ok = false;
             for (int q = 0; ok && q < n_active; ++q) {
                 const int a = down_slot(q, n_active, S), slot = q % nh;
-                if (q >= nh && !mbar_wait_sleepy(&hempty[slot], (uint32_t)((q / nh - 1) & 1), fa.err)) {
+                if (q >= nh && !mbar_wait_sleepy(&hempty[slot], (uint32_t)((q / nh - 1) & 1), fa.err, lim)) {
                     ok = false;
                     break;
                 }
@@ -1306,7 +1311,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
                             ready = 0;
                             break;
                         }
-                        if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+                        if (clock64() - t0 > lim) {
                             atomicExch(fa.err, ERR_TIMEOUT);
                             ready = 0;
                             break;
@@ -1363,7 +1368,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
             const ExpertDev ex = fa.experts[e];
             const float sg = __ldg(ex.gate.scales + c * 32 + lane);
             const float su = __ldg(ex.up.scales + c * 32 + lane);
-            if (!mbar_wait_sleepy(&ebars->part_full[buf], (uint32_t)((n >> 1) & 1), fa.err)) {
+            if (!mbar_wait_sleepy(&ebars->part_full[buf], (uint32_t)((n >> 1) & 1), fa.err, lim)) {
                 *abort = 1;
                 break;
             }
@@ -1481,7 +1486,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
                                  fa.xd + (int64_t)t * nbH);
     }
     named_bar(1, 256);
-    if (tid == 0) flags[0] = grid_barrier(fa.gbar, G, fa.err) ? 1 : 0;
+    if (tid == 0) flags[0] = grid_barrier(fa.gbar, G, fa.err, lim) ? 1 : 0;
     named_bar(1, 256);
     if (!flags[0]) {
         *abort = 1;
@@ -1555,14 +1560,14 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         const bool fast = geo.fast && (MAXT == 1 || ne == 1);
         LaneAct<BITS, 3> act;
         if (fast) act.load(acts + (size_t)tok[0] * rbH, H, V, fgeo.vbase);
-        if (n >= 2 && !mbar_wait(&ebars->part_free[buf], (uint32_t)(((n >> 1) - 1) & 1), fa.err)) {
+        if (n >= 2 && !mbar_wait(&ebars->part_free[buf], (uint32_t)(((n >> 1) - 1) & 1), fa.err, lim)) {
             ok = false;
             *abort = 1;
             break;
         }
         double *pbuf = part + (size_t)buf * 2 * part_mat;
         if (fast) {
-            const RingView rv{ring, bars, ns, fa.err, abort};
+            const RingView rv{ring, bars, ns, fa.err, abort, 1, lim};
             switch (fgeo.slices) {
                 case 1: ok = gateup_item_fast<BITS, 1>(rv, rp, RB, fgeo, act, pbuf, part_mat, ntok); break;
                 case 2: ok = gateup_item_fast<BITS, 2>(rv, rp, RB, fgeo, act, pbuf, part_mat, ntok); break;
@@ -1570,7 +1575,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
             }
         } else {
             for (int ms = 0; ms < steps; ++ms) {
-                if (!mbar_wait(&bars->full[rp.slot], rp.phase, fa.err)) {
+                if (!mbar_wait(&bars->full[rp.slot], rp.phase, fa.err, lim)) {
                     ok = false;
                     *abort = 1;
                     break;
@@ -1607,7 +1612,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
     // P4: down rows of every active expert as its h arrives, then the combine
     const int vpl = (VI % 32 == 0) ? VI / 32 : 0;
     DownLoop dl{lw.off, n_active, S, T, subs, ns, fa.down_rows, fa.rows_cap, r0, nrows, RBI, VI, I, rbI,
-                fa.down_span, ring, dscale, hslots, fa.nh, hfull, hempty, ebuf, bars, abort, fa.err};
+                fa.down_span, lim, ring, dscale, hslots, fa.nh, hfull, hempty, ebuf, bars, abort, fa.err};
     switch (vpl) {
         case 1: ok = down_loop<BITS, 1, MAXT>(dl, rp) && ok; break;
         case 2: ok = down_loop<BITS, 2, MAXT>(dl, rp) && ok; break;

@@ -112,6 +112,7 @@ struct TcArgs {
     float *hd;
     float *e_pairs;         // down output [pairs][H]
     int *err;
+    const long long *wait_limit;  // SM cycles a wait on progress may last (drains keep the default)
 };
 
 // --- tcgen05 wrappers -------------------------------------------------------
@@ -229,13 +230,14 @@ __global__ void k_pair_offsets(RouteWs ws, const int8_t *__restrict__ q, const f
 }
 
 // Bounded wait that also gives up once another role has aborted.
-__device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, TcBars *tb, int *err) {
+__device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, TcBars *tb, int *err,
+                                        long long lim) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*(volatile int *)&tb->abort) return false;
-        if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+        if (clock64() - t0 > lim) {
             atomicExch(err, ERR_TIMEOUT);
             *(volatile int *)&tb->abort = 1;
             return false;
@@ -299,6 +301,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_active = *a.ws.n_active;
+    const long long lim = *a.wait_limit;
     const TcLayout L = tc_layout(BITS, n_active);
     TcBars *tb = reinterpret_cast<TcBars *>(smem + L.bars);
     int *starts = reinterpret_cast<int *>(smem + L.starts);
@@ -406,7 +409,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
                 for (int s = 0; s < nstage; ++s, ++sc) {
                     const int slot = sc % TC_STAGES;
                     const uint32_t ph = (uint32_t)(sc / TC_STAGES) & 1u;
-                    if (!tc_wait(&tb->raw_empty[slot], ph ^ 1u, tb, a.err)) {
+                    if (!tc_wait(&tb->raw_empty[slot], ph ^ 1u, tb, a.err, lim)) {
                         ok = false;
                         break;
                     }
@@ -442,7 +445,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
             for (int s = 0; s < nstage && ok; ++s, ++sc) {
                 const int slot = sc % TC_STAGES;
-                if (!tc_wait(&tb->raw_full[slot], (uint32_t)(sc / TC_STAGES) & 1u, tb, a.err)) {
+                if (!tc_wait(&tb->raw_full[slot], (uint32_t)(sc / TC_STAGES) & 1u, tb, a.err, lim)) {
                     ok = false;
                     break;
                 }
@@ -452,8 +455,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
                 for (int j = 0; j < TC_BPS && ok; ++j, ++blk) {
                     if ((blk & 1) != grp) continue;
                     const int cs = blk % TC_SLOTS, db = blk % TC_BUFS;
-                    if (!tc_wait(&tb->op_empty[cs], ((uint32_t)(blk / TC_SLOTS) & 1u) ^ 1u, tb, a.err) ||
-                        !tc_wait(&tb->dd_empty[db], ((uint32_t)(blk / TC_BUFS) & 1u) ^ 1u, tb, a.err)) {
+                    if (!tc_wait(&tb->op_empty[cs], ((uint32_t)(blk / TC_SLOTS) & 1u) ^ 1u, tb, a.err, lim) ||
+                        !tc_wait(&tb->dd_empty[db], ((uint32_t)(blk / TC_BUFS) & 1u) ^ 1u, tb, a.err, lim)) {
                         ok = false;
                         break;
                     }
@@ -500,8 +503,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
                 for (int k = 0; k < nblk; ++k, ++blk) {
                     const int cs = blk % TC_SLOTS, bf = blk % TC_BUFS;
-                    if (!tc_wait(&tb->op_full[cs], (uint32_t)(blk / TC_SLOTS) & 1u, tb, a.err) ||
-                        !tc_wait(&tb->tm_empty[bf], ((uint32_t)(blk / TC_BUFS) & 1u) ^ 1u, tb, a.err)) {
+                    if (!tc_wait(&tb->op_full[cs], (uint32_t)(blk / TC_SLOTS) & 1u, tb, a.err, lim) ||
+                        !tc_wait(&tb->tm_empty[bf], ((uint32_t)(blk / TC_BUFS) & 1u) ^ 1u, tb, a.err, lim)) {
                         ok = false;
                         break;
                     }
@@ -540,7 +543,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
             for (int k = 0; k < nblk; ++k, ++blk) {
                 const int bf = blk % TC_BUFS;
                 const uint32_t ph = (uint32_t)(blk / TC_BUFS) & 1u;
-                if (!tc_wait(&tb->tm_full[bf], ph, tb, a.err)) {
+                if (!tc_wait(&tb->tm_full[bf], ph, tb, a.err, lim)) {
                     ok = false;
                     break;
                 }
@@ -550,7 +553,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_grouped_tc(const __grid_const
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tb->tm_empty[bf]);
-                if (!tc_wait(&tb->dd_full[bf], ph, tb, a.err)) {
+                if (!tc_wait(&tb->dd_full[bf], ph, tb, a.err, lim)) {
                     ok = false;
                     break;
                 }

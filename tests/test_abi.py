@@ -84,6 +84,7 @@ def test_argument_errors_need_no_device(L):
     assert L.coli_router(None, fake, 1, fake, fake, None) == qe.COLI_EINVAL
     assert L.coli_moe_forward(None, fake, 1, fake, None) == qe.COLI_EINVAL
     assert L.coli_dbg_block_sums(fake, 4, 1, 31, fake, 1, fake, None) == qe.COLI_EINVAL
+    assert L.coli_dbg_set_wait_limit(None, 100, None) == qe.COLI_EINVAL
     L.coli_moe_destroy(None)
 
 

@@ -191,6 +191,38 @@ def test_bounded_wait_reports_timeout_and_handle_recovers():
     gl.close()
 
 
+@pytest.mark.parametrize("path", ["decode", "tensor_cores"])
+def test_real_kernels_give_up_under_a_short_wait_limit(path):
+    """A short per-handle wait limit makes the waits inside the layer's own
+    kernels run out (the persistent decode kernel; the tcgen05 grouped GEMMs):
+    every forward then either completes or reports COLI_ETIMEOUT -- nothing
+    hangs or faults -- at least one reports it, and with the default limit
+    back the same handle computes the layer exactly as before."""
+    if path == "decode":
+        cfg = _small_cfg(hidden=384, inter=320, n_routed=16, n_group=4, topk_group=2, top_k=3,
+                         seed=11)
+        T = 4
+    else:
+        cfg = _small_cfg(hidden=512, inter=256, n_routed=16, n_group=4, topk_group=2, top_k=3,
+                         seed=12)
+        T = 37
+    gl = GpuLayer(cfg, max_tokens=T)
+    x = synth.tokens(cfg, T=T, device=DEV)
+    y0, _ = compare_forward(gl, x)
+    seen = []
+    for cycles in (100, 1000, 10000, 100000):
+        gl.handle.dbg_set_wait_limit(cycles)
+        gl.handle.forward(x)
+        seen.append(gl.handle.device_status())
+    gl.handle.dbg_set_wait_limit(0)
+    assert set(seen) <= {qe.COLI_OK, qe.COLI_ETIMEOUT}, seen
+    assert qe.COLI_ETIMEOUT in seen, seen
+    assert gl.handle.device_status() == qe.COLI_OK
+    y1, _ = compare_forward(gl, x)
+    np.testing.assert_array_equal(y0, y1)
+    gl.close()
+
+
 # ------------------------------------------------------- full-size workloads
 @pytest.fixture(scope="module")
 def glm52_layer():
