@@ -48,6 +48,12 @@ def lib():
         _LIB.oracle_route.argtypes = [vp, i64, i64, vp, vp, ci, ci, ci, ci, cf, vp, vp, vp, vp,
                                       vp, vp]
         _LIB.oracle_route.restype = ci
+        _LIB.oracle_fp8_e4m3.argtypes = [ctypes.c_uint8]
+        _LIB.oracle_fp8_e4m3.restype = cf
+        _LIB.oracle_dequant_fp8.argtypes = [vp, vp, i64, i64, i64, vp]
+        _LIB.oracle_dequant_fp8.restype = None
+        _LIB.oracle_requant_fp8.argtypes = [vp, vp, i64, i64, i64, ci, vp, vp]
+        _LIB.oracle_requant_fp8.restype = ci
         _LIB.oracle_swiglu.argtypes = [vp, vp, i64, vp]
         _LIB.oracle_swiglu.restype = None
         _LIB.oracle_expert.argtypes = [i64, i64, ci, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
@@ -146,6 +152,37 @@ def route(x, Wr, bias, top_k, n_group, topk_group, rsf):
         raise ValueError("oracle_route rejected E=%d G=%d gk=%d k=%d" % (E, n_group, topk_group,
                                                                         top_k))
     return dict(idx=idx, w=w, s=s, c=c, kmargin=km, gmargin=gm)
+
+
+def fp8_e4m3(code):
+    """Value of one FP8 e4m3 code (fp32; NaN for S.1111.111)."""
+    return float(lib().oracle_fp8_e4m3(int(code) & 0xFF))
+
+
+def dequant_fp8(codes, scale, block=128):
+    """FP8 codes [rows][K] (uint8) with block scales [ceil(rows/B)][ceil(K/B)]
+    -> fp32 weights [rows][K]."""
+    codes = _c(codes, np.uint8)
+    scale = _c(scale, np.float32)
+    rows, K = codes.shape
+    assert scale.shape == (-(-rows // block), -(-K // block))
+    out = np.empty((rows, K), np.float32)
+    lib().oracle_dequant_fp8(_p(codes), _p(scale), rows, K, block, _p(out))
+    return out
+
+
+def requant_fp8(codes, scale, bits, block=128):
+    """The converter step: FP8 + block scales -> per-row (codes, scales)."""
+    codes = _c(codes, np.uint8)
+    scale = _c(scale, np.float32)
+    rows, K = codes.shape
+    assert scale.shape == (-(-rows // block), -(-K // block))
+    out = np.empty((rows, row_bytes(K, bits)), np.uint8)
+    sc = np.empty(rows, np.float32)
+    rc = lib().oracle_requant_fp8(_p(codes), _p(scale), rows, K, block, bits, _p(out), _p(sc))
+    if rc != 0:
+        raise ValueError("oracle_requant_fp8 rc=%d" % rc)
+    return out, sc
 
 
 def swiglu(g, u):

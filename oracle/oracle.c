@@ -125,6 +125,48 @@ int oracle_quant_weights(const float *w, int64_t rows, int64_t K, int bits,
     return 0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* FP8 checkpoint weights.  [HN] 実装済みの主な機能, offline-converter bullet:
+ * the FP8 shards are dequantised with 128 x 128 block scales and then
+ * requantised into the engine's container (the per-row formats above).
+ * Reading (the pages name neither the FP8 variant nor the scale's
+ * direction): FP8 is e4m3 with no infinities -- 1 sign bit, 4 exponent bits
+ * with bias 7, 3 mantissa bits; exponent field 0 is subnormal
+ * (mantissa * 2^-9); the all-ones code S.1111.111 is NaN (so the largest
+ * magnitude is 448) -- and the block scale multiplies:
+ *   w[r][k] = (float)( e4m3(code[r][k]) * scale[r / B][k / B] )   (fp32)
+ * with the scale grid ceil(rows / B) x ceil(K / B) for block size B.  The
+ * requantised row is then oracle_quant_weights of these fp32 values. */
+float oracle_fp8_e4m3(uint8_t code)
+{
+    const int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    if (e == 15 && m == 7) return NAN;
+    double v = (e == 0) ? ldexp((double)m, -9) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return (float)(sign ? -v : v);
+}
+
+void oracle_dequant_fp8(const uint8_t *codes, const float *scale, int64_t rows, int64_t K,
+                        int64_t block, float *out)
+{
+    const int64_t kb = (K + block - 1) / block;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < K; ++k)
+            out[r * K + k] = oracle_fp8_e4m3(codes[r * K + k]) * scale[(r / block) * kb + k / block];
+}
+
+/* The whole converter step for one matrix: FP8 + block scales -> per-row
+ * int8 / int4 / int2 codes and scales.  Returns oracle_quant_weights's code. */
+int oracle_requant_fp8(const uint8_t *codes, const float *scale, int64_t rows, int64_t K,
+                       int64_t block, int bits, uint8_t *out_codes, float *out_scales)
+{
+    float *w = malloc(sizeof(float) * (size_t)(rows * K));
+    if (!w) return -2;
+    oracle_dequant_fp8(codes, scale, rows, K, block, w);
+    int rc = oracle_quant_weights(w, rows, K, bits, out_codes, out_scales);
+    free(w);
+    return rc;
+}
+
 /* Unpack codes back to signed integers (one int8 per element). */
 int oracle_unpack_weights(const uint8_t *codes, int64_t rows, int64_t K, int bits, int8_t *out)
 {

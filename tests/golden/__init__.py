@@ -97,5 +97,14 @@ def swiglu_expert():
     return out
 
 
-__all__ = ["q8_blocks", "weight_rows", "single_expert_y", "swiglu_cases", "swiglu_expert",
+def fp8_e4m3():
+    """[(code, value)] from fp8_e4m3.txt (value a Python float, nan allowed)."""
+    out = []
+    for ln in _lines("fp8_e4m3.txt"):
+        c, v = (t.strip() for t in ln.split("|"))
+        out.append((int(c, 16), float(v)))
+    return out
+
+
+__all__ = ["fp8_e4m3", "q8_blocks", "weight_rows", "single_expert_y", "swiglu_cases", "swiglu_expert",
            "Fraction"]

@@ -93,6 +93,59 @@ def test_weight_roundtrip(bits, qmax, lo, hi):
     np.testing.assert_array_equal(top, expect)
 
 
+# ------------------------------------------------------ FP8 checkpoint weights
+def test_fp8_e4m3_hand_values():
+    for code, value in golden.fp8_e4m3():
+        got = oracle.fp8_e4m3(code)
+        if math.isnan(value):
+            assert math.isnan(got), hex(code)
+        else:
+            assert got == value and math.copysign(1.0, got) == math.copysign(1.0, value), hex(code)
+
+
+def test_fp8_e4m3_all_codes_match_torch():
+    """Every one of the 256 codes decodes as torch's own float8_e4m3fn does."""
+    import torch
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    got = np.array([oracle.fp8_e4m3(c) for c in range(256)], np.float32)
+    nan = np.isnan(ref)
+    assert nan.sum() == 2 and np.array_equal(nan, np.isnan(got))
+    np.testing.assert_array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+
+
+def test_dequant_fp8_block_grid_on_ragged_shapes():
+    """Block (r // 128, k // 128) scales element (r, k), ragged last blocks
+    included: with every code 1.0 the output is the scale grid, block by block."""
+    rows, K = 130, 224
+    codes = np.full((rows, K), 0x38, np.uint8)          # 1.0
+    scale = np.array([[0.5, 2.0], [4.0, 0.25]], np.float32)
+    w = oracle.dequant_fp8(codes, scale, block=128)
+    assert np.all(w[:128, :128] == 0.5) and np.all(w[:128, 128:] == 2.0)
+    assert np.all(w[128:, :128] == 4.0) and np.all(w[128:, 128:] == 0.25)
+    # one code per block, negative and subnormal values
+    codes[0, 0], codes[129, 223], codes[5, 130] = 0xB8, 0x01, 0x7E
+    w = oracle.dequant_fp8(codes, scale, block=128)
+    assert w[0, 0] == -0.5 and w[129, 223] == np.float32(0.25 * 2.0 ** -9) and w[5, 130] == 896.0
+
+
+def test_requant_fp8_on_hand_rows():
+    """FP8 codes of the hand-computed weight rows (encoded by torch) with a
+    block scale of 1 requantise to the hand-computed per-row codes."""
+    import torch
+    tested = 0
+    for bits, w, s, q, by in golden.weight_rows():
+        enc = torch.from_numpy(w).to(torch.float8_e4m3fn)
+        if not torch.equal(enc.to(torch.float32), torch.from_numpy(w)):
+            continue  # a row e4m3 cannot hold exactly (e.g. 127)
+        codes = enc.view(torch.uint8).numpy()[None]
+        c, sc = oracle.requant_fp8(codes, np.ones((1, 1), np.float32), bits, block=128)
+        assert sc[0] == s
+        np.testing.assert_array_equal(c[0], by)
+        tested += 1
+    assert tested >= 2
+
+
 # -------------------------------------------------------------------- int dot
 def _rand_q8(K):
     x = RNG.standard_normal(K).astype(np.float32) * RNG.uniform(0.1, 5.0)
