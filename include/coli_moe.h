@@ -116,6 +116,23 @@ coli_status coli_quant_q8(const float *x, int64_t rows, int64_t len, int8_t *q, 
 coli_status coli_quant_weights(const float *w, int64_t rows, int64_t K, int wfmt, void *codes,
                                float *scales, coli_stream_t stream);
 
+/* FP8 checkpoint weights -> per-row weight format ([HN] 実装済みの主な機能,
+ * offline-converter bullet: the FP8 shards are dequantised with 128 x 128
+ * block scales, then requantised into the engine's container).
+ *   w_fp8 [rows][K] one e4m3 code per byte (1 sign, 4 exponent bits with
+ *     bias 7, 3 mantissa bits, no infinities, S.1111.111 NaN); device,
+ *     16-byte aligned;
+ *   block_scale [ceil(rows/block)][ceil(K/block)] fp32, device: the block's
+ *     multiplier, w = fp32(e4m3(code) * block_scale[r/block][k/block]);
+ *   block: a positive multiple of 16 (the checkpoints use 128);
+ *   -> codes [rows][K*wfmt/8], scales [rows] exactly as coli_quant_weights
+ *     of the dequantised rows.
+ *   K % 32 == 0 (K % 64 == 0 for COLI_W_INT2); rows == 0 is a no-op.  NaN
+ *   codes give unspecified (memory-safe) results. */
+coli_status coli_requant_fp8(const void *w_fp8, const float *block_scale, int64_t rows, int64_t K,
+                            int64_t block, int wfmt, void *codes, float *scales,
+                            coli_stream_t stream);
+
 /* Create a layer handle ([HN] router and batch-union bullets).
  *   router_w [E][H] fp32 and bias [E] fp32 (e_score_correction_bias) are
  *   device pointers; experts is a HOST array of E + S coli_expert records

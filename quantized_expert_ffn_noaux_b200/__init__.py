@@ -69,6 +69,7 @@ def lib():
         "coli_launch_count": ([], ctypes.c_uint64),
         "coli_quant_q8": ([vp, i64, i64, vp, vp, vp], ci),
         "coli_quant_weights": ([vp, i64, i64, ci, vp, vp, vp], ci),
+        "coli_requant_fp8": ([vp, vp, i64, i64, i64, ci, vp, vp, vp], ci),
         "coli_moe_create": ([vp, vp, vp, vp, ctypes.POINTER(vp)], ci),
         "coli_router": ([vp, vp, ci, vp, vp, vp], ci),
         "coli_moe_forward": ([vp, vp, ci, vp, vp], ci),
@@ -133,6 +134,19 @@ def quant_weights(w, bits, codes=None, scales=None, stream=None):
         scales = torch.empty(rows, dtype=torch.float32, device=w.device)
     _check(lib().coli_quant_weights(_ptr(w), rows, K, bits, _ptr(codes), _ptr(scales),
                                     _stream(stream)))
+    return codes, scales
+
+
+def requant_fp8(w_fp8, block_scale, bits, block=128, codes=None, scales=None, stream=None):
+    """FP8 e4m3 codes w_fp8 [rows][K] (uint8, device) with block scales
+    [ceil(rows/block)][ceil(K/block)] fp32 -> per-row (codes uint8, scales fp32)."""
+    rows, K = w_fp8.shape
+    if codes is None:
+        codes = torch.empty((rows, row_bytes(K, bits)), dtype=torch.uint8, device=w_fp8.device)
+    if scales is None:
+        scales = torch.empty(rows, dtype=torch.float32, device=w_fp8.device)
+    _check(lib().coli_requant_fp8(_ptr(w_fp8), _ptr(block_scale), rows, K, block, bits,
+                                  _ptr(codes), _ptr(scales), _stream(stream)))
     return codes, scales
 
 

@@ -870,6 +870,32 @@ coli_status coli_quant_weights(const float *w, int64_t rows, int64_t K, int wfmt
     return L.done();
 }
 
+coli_status coli_requant_fp8(const void *w_fp8, const float *block_scale, int64_t rows, int64_t K,
+                            int64_t block, int wfmt, void *codes, float *scales,
+                            coli_stream_t stream) {
+    g_last_error.clear();
+    if (wfmt != 8 && wfmt != 4 && wfmt != 2) return fail(COLI_EINVAL, "wfmt must be 8, 4 or 2");
+    if (rows < 0 || K <= 0 || K % (wfmt == 2 ? 64 : 32))
+        return fail(COLI_EINVAL, "K must be a positive multiple of 32 (64 for int2)");
+    if (block <= 0 || block % 16) return fail(COLI_EINVAL, "block must be a positive multiple of 16");
+    if (rows == 0) return COLI_OK;
+    if (!w_fp8 || !block_scale || !codes || !scales) return fail(COLI_EINVAL, "null pointer");
+    if (!aligned16(w_fp8) || !aligned16(codes) || !((uintptr_t)block_scale % 4 == 0) ||
+        !((uintptr_t)scales % 4 == 0))
+        return fail(COLI_EINVAL, "w_fp8 and codes must be 16-byte aligned, scales 4-byte aligned");
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t grid = std::min<int64_t>((rows + 7) / 8, (int64_t)sm_count() * 16);
+    const uint8_t *w8 = (const uint8_t *)w_fp8;
+    uint8_t *c = (uint8_t *)codes;
+    Launch L(nullptr, s, "requant_fp8");
+    switch (wfmt) {
+        case 8: k_requant_fp8<8><<<(unsigned)grid, 256, 0, s>>>(w8, block_scale, rows, K, block, c, scales); break;
+        case 4: k_requant_fp8<4><<<(unsigned)grid, 256, 0, s>>>(w8, block_scale, rows, K, block, c, scales); break;
+        default: k_requant_fp8<2><<<(unsigned)grid, 256, 0, s>>>(w8, block_scale, rows, K, block, c, scales); break;
+    }
+    return L.done();
+}
+
 size_t coli_moe_workspace_bytes(const coli_moe_config *cfg) {
     if (!cfg_valid(cfg, nullptr)) return 0;
     return layout_of(*cfg).total;
