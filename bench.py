@@ -57,6 +57,9 @@ def parse():
                    help="tokens in the CPU-baseline sample (default: one per host thread)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-graph", action="store_true")
+    p.add_argument("--no-prefill", action="store_true",
+                   help="skip the extra batch-union prefill measurement (2048 tokens)")
+    p.add_argument("--prefill-steps", type=int, default=10)
     return p.parse_args()
 
 
@@ -372,6 +375,70 @@ def run_coli(args, cfg, rank, world, device):
     return result, cpu
 
 
+def run_prefill(args, device):
+    """The batch-union prefill workload (2048 tokens through one layer of the
+    same shape; every expert is active): throughput and the bounds of its
+    dominant kernel, timed with CUDA events on the launching stream."""
+    import quantized_expert_ffn_noaux_b200 as qe
+    cfg = synth.workload("glm52_prefill_int4_t2048")
+    T = cfg["tokens"]
+    lay = build_layers(cfg, 1, T, device, qe)[0]
+    x = synth.tokens(cfg, T=T, device=device)
+    out = torch.empty_like(x)
+    stream = torch.cuda.Stream(device=device)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            lay.forward(x, out)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(args.prefill_steps):
+            lay.forward(x, out)
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / args.prefill_steps
+    lay.profile(True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            lay.forward(x, out)
+    torch.cuda.synchronize()
+    kt = lay.profile_read()
+    lay.profile(False)
+    lay.close()
+    H, I, E, S, k = cfg["hidden"], cfg["inter"], cfg["n_routed"], cfg["n_shared"], cfg["top_k"]
+    gu_b, dn_b = expert_bytes(cfg)
+    weight_bytes = (E + S) * (gu_b + dn_b)          # every expert is active at 2048 tokens
+    pairs = T * (k + S)
+    macs = pairs * 3 * H * I                        # gate, up, down
+    peak, peak_kind = peaks()
+    nsm = torch.cuda.get_device_properties(device).multi_processor_count
+    dom = max(kt.items(), key=lambda kv: kv[1][1])[0]
+    n_dom, ms_dom = kt[dom]
+    dom_ms = ms_dom / n_dom
+    blocks = pairs * 2 * I * (H // 32) if dom.startswith("gateup") else pairs * H * (I // 32)
+    dmacs = pairs * 2 * I * H if dom.startswith("gateup") else pairs * H * I
+    peak_fp64 = nsm * 64 * sm_max_mhz() * 1e6 / 1e9
+    ach = 2 * blocks / (dom_ms / 1e3) / 1e9
+    return {
+        "workload": cfg["name"], "tokens_per_step": T, "value": round(T / (ms / 1e3), 1),
+        "unit": "tokens/s", "ms_per_step": round(ms, 4), "steps": args.prefill_steps,
+        "expert_weight_gbs": round(weight_bytes / (ms / 1e3) / 1e9, 1),
+        "hbm_frac_of_step": round(weight_bytes / (ms / 1e3) / 1e9 / peak, 4),
+        "int8_tensor_tops": round(2 * macs / (ms / 1e3) / 1e12, 2),
+        "int8_tensor_frac_of_nominal_4500": round(2 * macs / (ms / 1e3) / 1e12 / 4500.0, 4),
+        "roofline": {"bound": "alu", "achieved": round(ach, 1), "peak": round(peak_fp64, 1),
+                     "unit": "Gop/s", "frac": round(ach / peak_fp64, 4), "kernel": dom,
+                     "ops": "fp64 promotion of 32-block int8 products: convert + FMA",
+                     "peak_source": "derived: %d SMs x 64 fp64 lanes x %.0f MHz" % (nsm, sm_max_mhz()),
+                     "avg_launch_ms": round(dom_ms, 4),
+                     "int8_tensor_tops": round(2 * dmacs / (dom_ms / 1e3) / 1e12, 2),
+                     "traffic": recorded_traffic(dom, cfg["name"])},
+        "hbm_peak": peak, "hbm_peak_source": peak_kind,
+        "kernels": {kname: {"launches": v[0], "ms": round(v[1], 3)} for kname, v in kt.items()},
+    }
+
+
 def oracle_layer_for(cfg, Wr, bias, needed, fp32_fn, threads):
     import oracle
     E, S = cfg["n_routed"], cfg["n_shared"]
@@ -512,6 +579,11 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
     res, cpu = run_coli(args, cfg, rank, world, device)
+    prefill = None
+    if world == 1 and not args.no_prefill and args.workload == "glm52_decode_int4_t1" \
+            and args.n_routed is None:
+        torch.cuda.empty_cache()
+        prefill = run_prefill(args, device)
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(res["value"], 2), "unit": "tokens/s",
@@ -533,6 +605,7 @@ def main():
             "union_experts_per_step": res["union_experts_per_step"],
             "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res["e2e"],
             "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
+            "prefill": prefill,
             "kernels": res["kernels"],
         }
         print(json.dumps(line), flush=True)

@@ -176,6 +176,36 @@ coli_status coli_moe_forward(coli_moe *m, const float *x, int T, float *out,
 coli_status coli_moe_forward_host(coli_moe *m, const float *x_host, int T, float *out_host,
                                   coli_stream_t stream);
 
+/* Expert parallelism over several GPUs (one handle per GPU): the layer's
+ * routed experts are split into contiguous ranges, one per GPU, the router
+ * is replicated and one GPU also computes the shared experts; every GPU's
+ * partial output covers the (token, expert) pairs it owns, and the partials
+ * are summed in a fixed GPU order.  ("Comment exécuter un réseau de neurones
+ * de 744 milliards de paramètres sur un ordinateur ordinaire", devtrends.cc,
+ * "Les chiffres réels de vitesse": six GPUs keep the experts entirely in
+ * video memory; the pages do not say how they are split.)
+ *
+ * coli_moe_set_experts: later forwards on this handle compute only routed
+ *   experts e_lo <= e < e_hi and, if own_shared, the shared experts (every
+ *   token still routes over all experts).  Expert weights outside the range
+ *   are never read, so they may be placeholders.  0 <= e_lo <= e_hi <= E.
+ *
+ * coli_moe_forward_partial: as coli_moe_forward, but writes the fp64 sum of
+ *   this handle's slots, unrounded, shared experts first and then routed
+ *   slots in order:  y_partial[t][r] = sum_{owned shared} e + sum_{owned j}
+ *   w[t][j] e_j  (device, [T][H] fp64, 16-byte aligned, not aliasing x).
+ *
+ * coli_combine_partials: out[i] = (float)(parts[0][i] + parts[1][i] + ...)
+ *   in fp64 in part order; parts is [n_parts][n] fp64 (device), out [n] fp32.
+ *   With one part holding every expert the result equals coli_moe_forward
+ *   bit for bit; with several it differs only in the association of the fp64
+ *   sum (the same for every call: deterministic). */
+coli_status coli_moe_set_experts(coli_moe *m, int e_lo, int e_hi, int own_shared);
+coli_status coli_moe_forward_partial(coli_moe *m, const float *x, int T, double *y_partial,
+                                     coli_stream_t stream);
+coli_status coli_combine_partials(const double *parts, int n_parts, int64_t n, float *out,
+                                  coli_stream_t stream);
+
 /* Release the handle and its workspace (not the borrowed weights).  Waits for
  * work already enqueued on the handle's last stream.  NULL is a no-op. */
 void coli_moe_destroy(coli_moe *m);

@@ -74,6 +74,9 @@ def lib():
         "coli_router": ([vp, vp, ci, vp, vp, vp], ci),
         "coli_moe_forward": ([vp, vp, ci, vp, vp], ci),
         "coli_moe_forward_host": ([vp, vp, ci, vp, vp], ci),
+        "coli_moe_set_experts": ([vp, ci, ci, ci], ci),
+        "coli_moe_forward_partial": ([vp, vp, ci, vp, vp], ci),
+        "coli_combine_partials": ([vp, ci, i64, vp, vp], ci),
         "coli_moe_destroy": ([vp], None),
         "coli_moe_workspace_bytes": ([vp], ctypes.c_size_t),
         "coli_moe_profile": ([vp, ci], ci),
@@ -252,6 +255,18 @@ class MoELayer:
         _check(lib().coli_moe_forward(self._h, _ptr(x), T, _ptr(out), _stream(stream)))
         return out
 
+    def set_experts(self, e_lo, e_hi, own_shared=True):
+        """Compute only routed experts [e_lo, e_hi) (and the shared ones if own_shared)."""
+        _check(lib().coli_moe_set_experts(self._h, int(e_lo), int(e_hi), 1 if own_shared else 0))
+
+    def forward_partial(self, x, out=None, stream=None):
+        """fp64 [T][H]: the unrounded sum over this handle's experts' slots."""
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty(x.shape, dtype=torch.float64, device=x.device)
+        _check(lib().coli_moe_forward_partial(self._h, _ptr(x), T, _ptr(out), _stream(stream)))
+        return out
+
     def forward_host(self, x_host, out_host, stream=None):
         """x_host, out_host: CPU fp32 tensors (pinned for async copies)."""
         T = x_host.shape[0]
@@ -290,3 +305,70 @@ class MoELayer:
         _check(lib().coli_dbg_last_forward(self._h, T, _ptr(idx), _ptr(w), _ptr(hq), _ptr(hd),
                                            _stream(stream)))
         return idx, w, hq, hd
+
+
+# ---------------------------------------------------------- expert parallelism
+def combine_partials(parts, out=None, stream=None):
+    """parts: fp64 [R][...] (device, part order) -> fp32 [...] = fp32(sum in part order)."""
+    n = parts[0].numel()
+    if out is None:
+        out = torch.empty(parts.shape[1:], dtype=torch.float32, device=parts.device)
+    _check(lib().coli_combine_partials(_ptr(parts), parts.shape[0], n, _ptr(out), _stream(stream)))
+    return out
+
+
+def expert_range(n_routed, rank, world):
+    """Contiguous routed-expert range [lo, hi) of `rank` among `world` GPUs,
+    sizes differing by at most one."""
+    base, rem = divmod(n_routed, world)
+    lo = rank * base + min(rank, rem)
+    return lo, lo + base + (1 if rank < rem else 0)
+
+
+def gather_partials(part, group=None):
+    """All ranks' partial outputs, stacked in rank order ([R][...]), on every rank."""
+    dist = torch.distributed
+    world = dist.get_world_size(group)
+    parts = [torch.empty_like(part) for _ in range(world)]
+    dist.all_gather(parts, part.contiguous(), group=group)
+    return torch.stack(parts)
+
+
+class ExpertParallelLayer:
+    """This GPU's share of an expert-parallel layer: the router (replicated),
+    routed experts expert_range(E, rank, world) and, on rank 0, the shared
+    experts.  forward() computes the fp64 partial over this rank's (token,
+    expert) pairs, all-gathers the partials over `group` (NCCL between GPUs)
+    and sums them in rank order on every rank: the same output on every rank,
+    deterministic from call to call.
+
+    experts: list of E + S Expert objects; those this rank does not own may be
+    None (a placeholder is passed; its weights are never read)."""
+
+    def __init__(self, cfg, router_w, bias, experts, rank, world, group=None):
+        self.rank, self.world, self.group = rank, world, group
+        self.e_lo, self.e_hi = expert_range(cfg["n_routed"], rank, world)
+        E = cfg["n_routed"]
+        dev = router_w.device
+        ph = None
+        full = []
+        for e, ex in enumerate(experts):
+            owned = (self.e_lo <= e < self.e_hi) if e < E else rank == 0
+            if ex is None:
+                if owned:
+                    raise ValueError("expert %d is owned by rank %d but not given" % (e, rank))
+                if ph is None:
+                    z = torch.zeros(16, dtype=torch.uint8, device=dev)
+                    sc = torch.zeros(4, dtype=torch.float32, device=dev)
+                    ph = Expert((z, sc), (z, sc), (z, sc))
+                ex = ph
+            full.append(ex)
+        self.layer = MoELayer(cfg, router_w, bias, full)
+        self.layer.set_experts(self.e_lo, self.e_hi, own_shared=(rank == 0))
+
+    def forward(self, x, stream=None):
+        part = self.layer.forward_partial(x, stream=stream)
+        return combine_partials(gather_partials(part, self.group), stream=stream)
+
+    def close(self):
+        self.layer.close()

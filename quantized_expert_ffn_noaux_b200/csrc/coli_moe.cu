@@ -108,6 +108,7 @@ struct coli_moe {
     unsigned long long *gbar = nullptr;
     int *hcnt = nullptr;  // per active expert: gate/up items done (decode kernel)
     long long *wait_limit = nullptr;  // SM cycles a kernel's wait on progress may last
+    double *out_partial = nullptr;    // set during coli_moe_forward_partial
     int last_T = 0;
     std::map<const void *, int> occ_cache;  // kernel -> CTAs per SM (attributes already set)
     // profiling
@@ -327,7 +328,7 @@ coli_status launch_down_small_t(coli_moe *m, int T, float *out, cudaStream_t s) 
     grid = std::max(grid, 1);
     Launch L(m, s, "down_combine");
     kern<<<grid, 256, smem, s>>>(m->rw, m->experts_dev, m->hq, m->hd, T, c.hidden, c.inter,
-                                 c.top_k, c.n_shared, out);
+                                 c.top_k, c.n_shared, out, m->out_partial);
     return L.done();
 }
 
@@ -563,6 +564,7 @@ coli_status launch_small_path(coli_moe *m, const float *x, int T, float *out, cu
     fa.hq = m->hq;
     fa.hd = m->hd;
     fa.out = out;
+    fa.out_partial = m->out_partial;
     fa.err = m->err;
     fa.wait_limit = m->wait_limit;
     fa.gbar = m->gbar;
@@ -701,7 +703,8 @@ coli_status launch_tc_path(coli_moe *m, int T, float *out, cudaStream_t s) {
     Launch L(m, s, "combine");
     const int64_t n = (int64_t)T * c.hidden;
     int grid = (int)std::min<int64_t>((n + 255) / 256, (int64_t)m->nsm * 8);
-    k_combine<<<grid, 256, 0, s>>>(m->rw, m->e_pairs, T, c.hidden, c.top_k, c.n_shared, out);
+    k_combine<<<grid, 256, 0, s>>>(m->rw, m->e_pairs, T, c.hidden, c.top_k, c.n_shared, out,
+                                   m->out_partial);
     return L.done();
 }
 
@@ -759,7 +762,8 @@ coli_status forward_impl(coli_moe *m, const float *x, int T, float *out, cudaStr
         Launch L(m, s, "combine");
         const int64_t n = (int64_t)T * c.hidden;
         int grid = (int)std::min<int64_t>((n + 255) / 256, (int64_t)m->nsm * 8);
-        k_combine<<<grid, 256, 0, s>>>(m->rw, m->e_pairs, T, c.hidden, c.top_k, c.n_shared, out);
+        k_combine<<<grid, 256, 0, s>>>(m->rw, m->e_pairs, T, c.hidden, c.top_k, c.n_shared, out,
+                                   m->out_partial);
         st = L.done();
         if (st != COLI_OK) return st;
     }
@@ -782,10 +786,23 @@ __global__ void k_gather_h(const int32_t *__restrict__ tok_pair, const int8_t *_
                            int8_t *__restrict__ hq_out, float *__restrict__ hd_out) {
     const int ts = blockIdx.x;  // (token, slot)
     if (ts >= T * slots) return;
-    const int p = tok_pair[ts];
+    const int p = tok_pair[ts];  // -1: an expert another handle computes (zeros here)
     for (int i = threadIdx.x; i < I; i += blockDim.x) {
-        if (hq_out) hq_out[(int64_t)ts * I + i] = hq[(int64_t)p * I + i];
-        if (hd_out && i < I / COLI_QBLK) hd_out[(int64_t)ts * (I / COLI_QBLK) + i] = hd[(int64_t)p * (I / COLI_QBLK) + i];
+        if (hq_out) hq_out[(int64_t)ts * I + i] = p < 0 ? (int8_t)0 : hq[(int64_t)p * I + i];
+        if (hd_out && i < I / COLI_QBLK)
+            hd_out[(int64_t)ts * (I / COLI_QBLK) + i] = p < 0 ? 0.0f : hd[(int64_t)p * (I / COLI_QBLK) + i];
+    }
+}
+
+// Sum of the partial outputs of expert-parallel handles, in part order:
+// out[i] = fp32( parts[0][i] + parts[1][i] + ... ), fp64 throughout.
+__global__ void k_sum_partials(const double *__restrict__ parts, int n_parts, int64_t n,
+                               float *__restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        double acc = 0.0;
+        for (int r = 0; r < n_parts; ++r) acc += parts[(int64_t)r * n + i];
+        out[i] = (float)acc;
     }
 }
 
@@ -958,6 +975,9 @@ coli_status coli_moe_create(const coli_moe_config *cfg, const float *router_w, c
     m->rw.pair_slot = (int32_t *)(b + o.pair_slot);
     m->rw.tok_pair = (int32_t *)(b + o.tok_pair);
     m->rw.wstride = (cfg->max_tokens + 31) / 32;
+    m->rw.e_lo = 0;  // every routed and shared expert, until coli_moe_set_experts
+    m->rw.e_hi = cfg->n_routed;
+    m->rw.own_shared = 1;
     m->xq = (int8_t *)(b + o.xq);
     m->xd = (float *)(b + o.xd);
     m->hq = (int8_t *)(b + o.hq);
@@ -1041,6 +1061,49 @@ coli_status coli_moe_forward(coli_moe *m, const float *x, int T, float *out, col
     const char *xa = (const char *)x, *oa = (const char *)out;
     if (xa < oa + bytes && oa < xa + bytes) return fail(COLI_EINVAL, "out must not alias x");
     return forward_impl(m, x, T, out, (cudaStream_t)stream);
+}
+
+coli_status coli_moe_set_experts(coli_moe *m, int e_lo, int e_hi, int own_shared) {
+    g_last_error.clear();
+    coli_status st = check_handle(m);
+    if (st != COLI_OK) return st;
+    if (e_lo < 0 || e_hi < e_lo || e_hi > m->cfg.n_routed)
+        return fail(COLI_EINVAL, "expert range [%d, %d) outside [0, %d]", e_lo, e_hi, m->cfg.n_routed);
+    m->rw.e_lo = e_lo;
+    m->rw.e_hi = e_hi;
+    m->rw.own_shared = own_shared ? 1 : 0;
+    return COLI_OK;
+}
+
+coli_status coli_moe_forward_partial(coli_moe *m, const float *x, int T, double *y_partial,
+                                     coli_stream_t stream) {
+    g_last_error.clear();
+    coli_status st = check_handle(m);
+    if (st != COLI_OK) return st;
+    if (T < 1 || T > m->cfg.max_tokens) return fail(COLI_EINVAL, "T=%d outside [1, max_tokens=%d]", T, m->cfg.max_tokens);
+    if (!x || !y_partial) return fail(COLI_EINVAL, "null pointer");
+    if (!aligned16(x) || !aligned16(y_partial)) return fail(COLI_EINVAL, "pointers must be 16-byte aligned");
+    const size_t xb = (size_t)T * m->cfg.hidden * 4, yb = 2 * xb;
+    const char *xa = (const char *)x, *ya = (const char *)y_partial;
+    if (xa < ya + yb && ya < xa + xb) return fail(COLI_EINVAL, "y_partial must not alias x");
+    m->out_partial = y_partial;
+    st = forward_impl(m, x, T, nullptr, (cudaStream_t)stream);
+    m->out_partial = nullptr;
+    return st;
+}
+
+coli_status coli_combine_partials(const double *parts, int n_parts, int64_t n, float *out,
+                                  coli_stream_t stream) {
+    g_last_error.clear();
+    if (n_parts < 1 || n < 0) return fail(COLI_EINVAL, "n_parts must be >= 1 and n >= 0");
+    if (n == 0) return COLI_OK;
+    if (!parts || !out) return fail(COLI_EINVAL, "null pointer");
+    if (!aligned16(parts) || !aligned16(out)) return fail(COLI_EINVAL, "pointers must be 16-byte aligned");
+    cudaStream_t s = (cudaStream_t)stream;
+    const int grid = (int)std::min<int64_t>((n + 255) / 256, (int64_t)sm_count() * 8);
+    Launch L(nullptr, s, "sum_partials");
+    k_sum_partials<<<grid, 256, 0, s>>>(parts, n_parts, n, out);
+    return L.done();
 }
 
 coli_status coli_moe_forward_host(coli_moe *m, const float *x_host, int T, float *out_host,

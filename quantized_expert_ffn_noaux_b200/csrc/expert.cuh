@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(256) k_down_grouped(RouteWs ws,
 // Combine for many tokens: out[t][r] = fp64 sum, shared experts first, then
 // routed slots in order, of weight * e (weight 1 for shared experts).
 __global__ void k_combine(RouteWs ws, const float *__restrict__ e_pairs, int T, int H, int k,
-                          int S, float *__restrict__ out) {
+                          int S, float *__restrict__ out, double *__restrict__ out_partial) {
     const int64_t n = (int64_t)T * H;
     const int slots = k + S;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
@@ -268,13 +268,17 @@ __global__ void k_combine(RouteWs ws, const float *__restrict__ e_pairs, int T, 
         for (int jj = 0; jj < slots; ++jj) {
             const int j = jj < S ? k + jj : jj - S;
             const int p = ws.tok_pair[(int64_t)t * slots + j];
+            if (p < 0) continue;  // an expert another handle computes
             const double ev = (double)e_pairs[(int64_t)p * H + r];
             if (j < k)
                 acc = fma((double)ws.w[(int64_t)t * k + j], ev, acc);
             else
                 acc += ev;
         }
-        out[i] = (float)acc;
+        if (out_partial)
+            out_partial[i] = acc;
+        else
+            out[i] = (float)acc;
     }
 }
 
@@ -289,7 +293,8 @@ __global__ void __launch_bounds__(256) k_down_combine(RouteWs ws,
                                                       const int8_t *__restrict__ hq,
                                                       const float *__restrict__ hd, int T, int H,
                                                       int I, int k, int S,
-                                                      float *__restrict__ out) {
+                                                      float *__restrict__ out,
+                                                      double *__restrict__ out_partial) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_active = *ws.n_active;
@@ -376,13 +381,17 @@ __global__ void __launch_bounds__(256) k_down_combine(RouteWs ws,
             for (int jj = 0; jj < slots; ++jj) {
                 const int j = jj < S ? k + jj : jj - S;
                 const int p = ws.tok_pair[(int64_t)t * slots + j];
+                if (p < 0) continue;  // an expert another handle computes
                 const double ev = ep[(size_t)p * DOWN_ROWS + rr];
                 if (j < k)
                     acc = fma((double)ws.w[(int64_t)t * k + j], ev, acc);
                 else
                     acc += ev;
             }
-            out[(int64_t)t * H + r0 + rr] = (float)acc;
+            if (out_partial)
+                out_partial[(int64_t)t * H + r0 + rr] = acc;
+            else
+                out[(int64_t)t * H + r0 + rr] = (float)acc;
         }
         __syncwarp();
     }
@@ -851,6 +860,7 @@ struct DecodeArgs {
     int8_t *hq;
     float *hd;
     float *out;
+    double *out_partial;        // if set: the unrounded fp64 sum of this handle's slots instead of out
     int *err;
     unsigned long long *gbar;   // grid-barrier arrival counter
     int *hcnt;                  // per active expert: gate/up items whose h records are written
@@ -1084,6 +1094,8 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
     EpiBars *ebars = reinterpret_cast<EpiBars *>(smem + sizeof(PipeBars) + 8);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int T = fa.T, H = fa.H, I = fa.I, E = fa.E, S = fa.S, k = fa.k;
+    // shared experts in the active list (the slot layout always has S of them)
+    const int Sa = fa.ws.shared_active(S);
     const int RB = H * BITS / 8, V = H * BITS / 128;
     const int RBI = I * BITS / 8, VI = I * BITS / 128;
     const GuGeom geo = gu_geometry(H, BITS);
@@ -1140,12 +1152,12 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
     pipe_init(bars, ns);
     __syncthreads();
     volatile int *abort = &bars->abort;
-    const int n_shared_items = S * nchunk;
+    const int n_shared_items = Sa * nchunk;
     auto item_of = [&](int j) { return (int)blockIdx.x + j * G; };
     auto item_expert_chunk = [&](int item, int n_active, int &a, int &e, int &c) {
         if (item < n_shared_items) {
             const int q = item / nchunk;
-            a = n_active - S + q;
+            a = n_active - Sa + q;
             e = E + q;
             c = item - q * nchunk;
         } else {
@@ -1197,7 +1209,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
                 bulk_prefetch_l2((c2.m < spm ? ex.gate.codes : ex.up.codes) + (size_t)row0 * RB, (uint32_t)gu_bytes);
                 c2.next(1 << 30, steps, subs);
             }
-            for (int i = 0; i < S; ++i)
+            for (int i = 0; i < Sa; ++i)
                 bulk_prefetch_l2(fa.experts[E + i].down.codes + (size_t)r0 * RBI, (uint32_t)(nrows * RBI));
         }
         __syncwarp();
@@ -1245,7 +1257,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
             const int rs = r0 + c.sb * fa.down_rows;
             const int nr = min(fa.down_rows, r0 + nrows - rs);
             bytes = (uint32_t)(nr * RBI);
-            return ptab[3 * down_slot(c.a, n_active, S) + 2] + (size_t)rs * RBI;
+            return ptab[3 * down_slot(c.a, n_active, Sa) + 2] + (size_t)rs * RBI;
         };
         // No L2 prefetch ahead of the ring: the bulk-copy unit of the SM is
         // what limits the issue rate, and a prefetch costs it as much as the
@@ -1296,7 +1308,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
             // slots in the x records' space: only once every consumer warp is done with them
             if (fa.h_alias && !mbar_wait_sleepy(xfree, 0, fa.err, lim)) ok = false;
             for (int q = 0; ok && q < n_active; ++q) {
-                const int a = down_slot(q, n_active, S), slot = q % nh;
+                const int a = down_slot(q, n_active, Sa), slot = q % nh;
                 if (q >= nh && !mbar_wait_sleepy(&hempty[slot], (uint32_t)((q / nh - 1) & 1), fa.err, lim)) {
                     ok = false;
                     break;
@@ -1611,7 +1623,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
     if (consumers_aborted(abort, flags + 1)) return;
     // P4: down rows of every active expert as its h arrives, then the combine
     const int vpl = (VI % 32 == 0) ? VI / 32 : 0;
-    DownLoop dl{lw.off, n_active, S, T, subs, ns, fa.down_rows, fa.rows_cap, r0, nrows, RBI, VI, I, rbI,
+    DownLoop dl{lw.off, n_active, Sa, T, subs, ns, fa.down_rows, fa.rows_cap, r0, nrows, RBI, VI, I, rbI,
                 fa.down_span, lim, ring, dscale, hslots, fa.nh, hfull, hempty, ebuf, bars, abort, fa.err};
     switch (vpl) {
         case 1: ok = down_loop<BITS, 1, MAXT>(dl, rp) && ok; break;
@@ -1627,13 +1639,17 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         for (int jj = 0; jj < slots; ++jj) {
             const int j = jj < S ? k + jj : jj - S;
             const int p = lw.tok_pair[t * slots + j];
+            if (p < 0) continue;  // an expert another handle computes
             const double ev = (double)ebuf[(size_t)p * fa.rows_cap + row];
             if (j < k)
                 acc = fma((double)w_s[t * k + j], ev, acc);
             else
                 acc += ev;
         }
-        fa.out[(int64_t)t * H + r0 + row] = (float)acc;
+        if (fa.out_partial)
+            fa.out_partial[(int64_t)t * H + r0 + row] = acc;
+        else
+            fa.out[(int64_t)t * H + r0 + row] = (float)acc;
     }
 }
 

@@ -25,8 +25,13 @@ struct RouteWs {
     int32_t *act_of;          // [E+S] active slot of each expert (-1 if none)
     int32_t *pair_tok;        // [Pmax] token of each pair
     int32_t *pair_slot;       // [Pmax] slot of each pair
-    int32_t *tok_pair;        // [T][k+S] pair of each (token, slot)
+    int32_t *tok_pair;        // [T][k+S] pair of each (token, slot); -1: expert not owned here
     int wstride;              // bitmap words per expert
+    // expert parallelism: this handle computes routed experts [e_lo, e_hi)
+    // and, if own_shared, the shared experts; the batch union holds only those
+    int e_lo, e_hi, own_shared;
+    __host__ __device__ bool owns(int e) const { return e >= e_lo && e < e_hi; }
+    __host__ __device__ int shared_active(int S) const { return own_shared ? S : 0; }
 };
 
 // ---------------------------------------------------------------------------
@@ -426,10 +431,17 @@ __device__ void warp_union_one(RouteWs ws, int E, int S, int k, const int *idx /
     const int lane = threadIdx.x & 31;
     for (int e = lane; e < E + S; e += 32) ws.act_of[e] = -1;
     __syncwarp();
+    // the selected experts this handle owns, ascending
+    int nk = 0;
+    for (int i = 0; i < k; ++i) nk += ws.owns(idx[i]);
     for (int j = lane; j < k; j += 32) {
         const int e = idx[j];
+        if (!ws.owns(e)) {
+            ws.tok_pair[j] = -1;
+            continue;
+        }
         int a = 0;
-        for (int i = 0; i < k; ++i) a += idx[i] < e;
+        for (int i = 0; i < k; ++i) a += ws.owns(idx[i]) && idx[i] < e;
         ws.active[a] = e;
         ws.off[a] = a;
         ws.act_of[e] = a;
@@ -437,8 +449,13 @@ __device__ void warp_union_one(RouteWs ws, int E, int S, int k, const int *idx /
         ws.pair_slot[a] = j;
         ws.tok_pair[j] = a;
     }
+    const int sa = ws.shared_active(S);
     for (int i = lane; i < S; i += 32) {
-        const int a = k + i;
+        if (i >= sa) {
+            ws.tok_pair[k + i] = -1;
+            continue;
+        }
+        const int a = nk + i;
         ws.active[a] = E + i;
         ws.off[a] = a;
         ws.act_of[E + i] = a;
@@ -447,8 +464,8 @@ __device__ void warp_union_one(RouteWs ws, int E, int S, int k, const int *idx /
         ws.tok_pair[k + i] = a;
     }
     if (lane == 0) {
-        ws.off[k + S] = k + S;
-        *ws.n_active = k + S;
+        ws.off[nk + sa] = nk + sa;
+        *ws.n_active = nk + sa;
     }
     __syncwarp();
 }
@@ -469,7 +486,8 @@ __global__ void __launch_bounds__(256) k_route_select(
     double *c_s = sm.c;
     const int *sel = idx_out + (int64_t)t * k;
     if (!do_union) return;
-    if (tid < k) atomicOr(ws.bitmap + (int64_t)sel[tid] * ws.wstride + (t >> 5), 1u << (t & 31));
+    if (tid < k && ws.owns(sel[tid]))
+        atomicOr(ws.bitmap + (int64_t)sel[tid] * ws.wstride + (t >> 5), 1u << (t & 31));
     __threadfence();
     __syncthreads();
     if (tid == 0) is_last = (atomicAdd(ws.counter, 1u) == (unsigned)(gridDim.x - 1));
@@ -510,20 +528,29 @@ __global__ void __launch_bounds__(256) k_route_select(
         na_base += ftot;
         pair_base += ctot;
     }
+    const int sa = ws.shared_active(S);
     for (int i = tid; i < S; i += 256) {
-        ws.active[na_base + i] = E + i;
-        ws.off[na_base + i] = pair_base + i * T;
-        ws.act_of[E + i] = na_base + i;
+        if (i < sa) {
+            ws.active[na_base + i] = E + i;
+            ws.off[na_base + i] = pair_base + i * T;
+            ws.act_of[E + i] = na_base + i;
+        } else {
+            ws.act_of[E + i] = -1;
+        }
     }
     if (tid == 0) {
-        ws.off[na_base + S] = pair_base + S * T;
-        *ws.n_active = na_base + S;
+        ws.off[na_base + sa] = pair_base + sa * T;
+        *ws.n_active = na_base + sa;
     }
     __syncthreads();
     const int slots = k + S;
     for (int i = tid; i < T * k; i += 256) {
         int tt = i / k, j = i % k;
         int e = __ldcg(idx_out + i);
+        if (!ws.owns(e)) {
+            ws.tok_pair[(int64_t)tt * slots + j] = -1;
+            continue;
+        }
         int64_t wo = (int64_t)e * ws.wstride + (tt >> 5);
         int rank = ws.prefix[wo] + __popc(__ldcg(ws.bitmap + wo) & ((1u << (tt & 31)) - 1u));
         int p = ws.off[ws.act_of[e]] + rank;
@@ -533,6 +560,10 @@ __global__ void __launch_bounds__(256) k_route_select(
     }
     for (int i = tid; i < T * S; i += 256) {
         int tt = i % T, sh = i / T;
+        if (sh >= sa) {
+            ws.tok_pair[(int64_t)tt * slots + k + sh] = -1;
+            continue;
+        }
         int p = ws.off[na_base + sh] + tt;
         ws.pair_tok[p] = tt;
         ws.pair_slot[p] = k + sh;
@@ -554,9 +585,12 @@ __device__ void cta_union_small(RouteWs ws, int T, int E, int S, int k,
     const int tid = threadIdx.x;
     for (int e = tid; e < E; e += 256) {
         int c = 0;
-        for (int i = 0; i < T * k; ++i) c += (idx[i] == e);
+        if (ws.owns(e))
+            for (int i = 0; i < T * k; ++i) c += (idx[i] == e);
         cnt[e] = c;
     }
+    // slots of experts this handle does not own stay -1
+    for (int i = tid; i < T * (k + S); i += 256) ws.tok_pair[i] = -1;
     Sync::sync();
     int na_base = 0, pair_base = 0;
     for (int e0 = 0; e0 < E; e0 += 256) {
@@ -588,7 +622,12 @@ __device__ void cta_union_small(RouteWs ws, int T, int E, int S, int k,
         na_base += ftot;
         pair_base += ctot;
     }
+    const int sa = ws.shared_active(S);
     for (int i = tid; i < S; i += 256) {
+        if (i >= sa) {
+            ws.act_of[E + i] = -1;
+            continue;
+        }
         const int a = na_base + i;
         ws.active[a] = E + i;
         ws.off[a] = pair_base + i * T;
@@ -601,8 +640,8 @@ __device__ void cta_union_small(RouteWs ws, int T, int E, int S, int k,
         }
     }
     if (tid == 0) {
-        ws.off[na_base + S] = pair_base + S * T;
-        *ws.n_active = na_base + S;
+        ws.off[na_base + sa] = pair_base + sa * T;
+        *ws.n_active = na_base + sa;
     }
 }
 
