@@ -446,6 +446,10 @@ int oracle_expert(int64_t H, int64_t I, int bits, const oracle_qmat *gate, const
  * (token, slot); slot j < k is routed slot j, slot k+i is shared expert i.
  * Outputs idx_out/w_out/hq_out/hd_out may be NULL.  nthreads > 1 splits the
  * tokens over OpenMP threads; the arithmetic per token does not change.
+ *
+ * A dense layer ([HN] router bullet: the first three layers are dense) is
+ * n_routed = 0 with top_k = 0: no routing, every token through the shared
+ * experts only (weight 1), y_t = (float)(sum of the shared experts' e).
  * Returns 0, -1 on invalid parameters, -3 if a needed expert is NULL. */
 int oracle_moe_forward(const oracle_cfg *cfg, const float *Wr, const float *bias,
                        const oracle_qmat *mats, const float *x, int64_t T,
@@ -458,7 +462,8 @@ int oracle_moe_forward(const oracle_cfg *cfg, const float *Wr, const float *bias
     const int G = cfg->n_group, gk = cfg->topk_group, bits = cfg->bits;
     if (H % QBLK || I % QBLK || S < 0) return -1;
     if (bits != 8 && bits != 4 && bits != 2) return -1;
-    if (!route_params_ok(E, G, gk, k)) return -1;
+    const int dense = E == 0 && k == 0;
+    if (dense ? S < 1 : !route_params_ok(E, G, gk, k)) return -1;
     const int slots = k + S;
 
     int32_t *idx = malloc(sizeof(int32_t) * (size_t)(T * k));
@@ -467,8 +472,8 @@ int oracle_moe_forward(const oracle_cfg *cfg, const float *Wr, const float *bias
     float *xd = malloc(sizeof(float) * (size_t)(T * (H / QBLK)));
     if (!idx || !w || !xq || !xd) { free(idx); free(w); free(xq); free(xd); return -2; }
 
-    /* 1. routing */
-    {
+    /* 1. routing (none in a dense layer) */
+    if (!dense) {
         double *s = malloc(sizeof(double) * E), *c = malloc(sizeof(double) * E);
         double *gs = malloc(sizeof(double) * G);
         unsigned char *gkeep = malloc(G), *taken = malloc(E);

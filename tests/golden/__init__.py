@@ -89,7 +89,7 @@ def swiglu_expert():
             d[key.strip()] = val.split()
     out = {name: np.array([m[r] for r in range(len(m))], np.float32) for name, m in rows.items()}
     out["x"] = np.array([[float(v) for v in d["x"]]], np.float32)
-    for k in ("g", "u", "h", "y"):
+    for k in ("g", "u", "h", "y", "e"):
         out[k] = np.array([float(v) for v in d[k]], np.float32)
     out["hq"] = np.array([int(v) for v in d["hq"]], np.int8)
     out["hd"] = np.float32(float(d["hd"][0]))

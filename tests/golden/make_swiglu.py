@@ -27,7 +27,8 @@ evaluation accurate to fp64 rounds to the same fp32 h.
 
 swiglu_expert.txt: one expert (hidden 32, intermediate 32, int4, power-of-two
 row scales) on one token, chosen so that g and u are exact fp32 values with
-|g| < 4; the expected Q8_0(h) codes and scale and the layer output y.
+|g| < 4; the expected Q8_0(h) codes and scale, the expert output e (a dense
+layer's output) and the layer output y.
 """
 import os
 import random
@@ -183,6 +184,7 @@ def make_expert():
     hq, hd = q8_block(h)
     down = [[Fraction(0)] * I for _ in range(H)]
     y = []
+    ev = []
     rsf = Fraction(3, 2)
     for r in range(H):
         kd = rnd.choice((4, 5, 6))
@@ -192,9 +194,10 @@ def make_expert():
             down[r][i] = Fraction(codes[i]) / _exp2(kd)
         S = sum(codes[i] * hq[i] for i in range(I))
         e = f32(S * hd / _exp2(kd))           # one block: S * d_h * row scale
+        ev.append(e)
         y.append(f32(rsf * e))                 # combine: w = rsf * s / s
     return dict(H=H, I=I, x=x, gate=gate, up=up, down=down, g=g, u=u, h=h, hq=hq, hd=hd,
-                y=y, rsf=rsf)
+                y=y, e=ev, rsf=rsf)
 
 
 def write():
@@ -223,6 +226,8 @@ def write():
         f.write("hq: %s\n" % " ".join(str(v) for v in ex["hq"]))
         f.write("hd: %s\n" % fmt(ex["hd"]))
         f.write("y: %s\n" % " ".join(fmt(v) for v in ex["y"]))
+        f.write("# e: the expert's output before the combine (a dense layer's output)\n")
+        f.write("e: %s\n" % " ".join(fmt(v) for v in ex["e"]))
 
 
 if __name__ == "__main__":

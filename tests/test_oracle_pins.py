@@ -410,6 +410,30 @@ def test_swiglu_expert_exact():
     np.testing.assert_array_equal(res["out"][0], ex["y"])
 
 
+def test_dense_layer_hand_computed():
+    """A dense layer (no router, the expert as its one shared expert, weight 1)
+    on the exact unsaturated expert outputs the expert's exact e."""
+    ex = golden.swiglu_expert()
+    H = I = 32
+    q = oracle.QExpert.quantise(ex["gate"], ex["up"], ex["down"], 4)
+    cfg = _cfg(hidden=H, inter=I, n_routed=0, n_shared=1, top_k=0)
+    layer = oracle.Layer(cfg, np.zeros((0, H), np.float32), np.zeros(0, np.float32), [q])
+    res = layer.forward(ex["x"])
+    np.testing.assert_array_equal(res["out"][0], ex["e"])
+    np.testing.assert_array_equal(res["hq"][0, 0], ex["hq"])
+
+
+def test_dense_layer_equals_moe_without_routed_weight():
+    """Dense layer == the same shared expert inside a MoE layer whose routed
+    weights are all zero (routed_scaling_factor 0), bit for bit."""
+    rng = np.random.default_rng(21)
+    moe = _layer(_cfg(n_routed=4, top_k=2, routed_scaling_factor=0.0), rng)
+    x = rng.standard_normal((5, 64)).astype(np.float32)
+    dense = oracle.Layer(_cfg(n_routed=0, top_k=0), np.zeros((0, 64), np.float32),
+                         np.zeros(0, np.float32), [moe.experts[-1]])
+    np.testing.assert_array_equal(dense.forward(x)["out"], moe.forward(x)["out"])
+
+
 def test_dense_mixture_when_k_equals_E():
     """top_k = E with one group: every expert is used with weight
     rsf * s_i / sum(s), so y = e_shared + rsf * sum_i (s_i / sum s) e_i."""
