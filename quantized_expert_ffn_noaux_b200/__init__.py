@@ -205,6 +205,8 @@ class MoELayer:
     routed_scaling_factor, bits, max_tokens.  router_w [E][H] and bias [E] are
     fp32 device tensors; experts is a list of E + S Expert (shared last).  The
     handle borrows all of them; this object keeps references so they outlive it.
+    A dense layer is n_routed = 0 with top_k = 0 (router_w and bias may be
+    None or empty): every token through the shared experts only.
     """
 
     def __init__(self, cfg, router_w, bias, experts):
@@ -221,7 +223,7 @@ class MoELayer:
         _check(lib().coli_moe_create(ctypes.byref(c), _ptr(router_w), _ptr(bias), arr,
                                      ctypes.byref(h)))
         self._h = h
-        self.device = router_w.device
+        self.device = router_w.device if router_w is not None else experts[0].gate[0].device
 
     def close(self):
         if getattr(self, "_h", None) and self._h.value:

@@ -148,8 +148,15 @@ bool cfg_valid(const coli_moe_config *c, std::string *why) {
         return bad("hidden must be a positive multiple of 32 (64 for int2), <= 16384");
     if (c->inter <= 0 || c->inter % q || c->inter > 16384)
         return bad("inter must be a positive multiple of 32 (64 for int2), <= 16384");
-    if (c->n_routed < 1 || c->n_routed > 1024) return bad("n_routed must be in [1, 1024]");
+    if (c->n_routed < 0 || c->n_routed > 1024) return bad("n_routed must be in [0, 1024]");
     if (c->n_shared < 0 || c->n_shared > 4) return bad("n_shared must be in [0, 4]");
+    if (c->n_routed == 0) {  // a dense layer: no router, shared experts only
+        if (c->top_k != 0 || c->n_shared < 1)
+            return bad("a layer without routed experts needs top_k = 0 and n_shared >= 1");
+        if (!(c->routed_scaling_factor == c->routed_scaling_factor)) return bad("routed_scaling_factor is NaN");
+        if (c->max_tokens < 1 || c->max_tokens > (1 << 20)) return bad("max_tokens must be in [1, 2^20]");
+        return true;
+    }
     if (c->n_group < 1 || c->n_routed % c->n_group) return bad("n_group must divide n_routed");
     if (c->topk_group < 1 || c->topk_group > c->n_group) return bad("topk_group must be in [1, n_group]");
     const int cand = c->topk_group * (c->n_routed / c->n_group);
@@ -501,7 +508,7 @@ coli_status launch_route(coli_moe *m, const float *x, int T, int32_t *idx, float
                                   nullptr, nullptr, 0, idx, w);
         return L.done();
     }
-    {
+    if (E > 0) {
         Launch L(m, s, "router_logits");
         if (T <= 8) {
             const int grid = (E + 7) / 8;
@@ -925,7 +932,8 @@ coli_status coli_moe_create(const coli_moe_config *cfg, const float *router_w, c
     *out = nullptr;
     std::string why;
     if (!cfg_valid(cfg, &why)) return fail(COLI_EINVAL, "invalid config: %s", why.c_str());
-    if (!router_w || !bias || !experts) return fail(COLI_EINVAL, "null router/bias/experts");
+    if (!experts || (cfg->n_routed > 0 && (!router_w || !bias)))
+        return fail(COLI_EINVAL, "null router/bias/experts");
     if (!aligned16(router_w) || !aligned16(bias)) return fail(COLI_EINVAL, "router pointers must be 16-byte aligned");
     const int n = cfg->n_routed + cfg->n_shared;
     std::vector<ExpertDev> host(n);
@@ -1047,6 +1055,7 @@ coli_status coli_router(coli_moe *m, const float *x, int T, int32_t *idx, float 
     if (T < 1 || T > m->cfg.max_tokens) return fail(COLI_EINVAL, "T=%d outside [1, max_tokens=%d]", T, m->cfg.max_tokens);
     if (!x || !idx || !w) return fail(COLI_EINVAL, "null pointer");
     if (!aligned16(x) || !aligned16(idx) || !aligned16(w)) return fail(COLI_EINVAL, "pointers must be 16-byte aligned");
+    if (m->cfg.n_routed == 0) return fail(COLI_EINVAL, "a dense layer has no router");
     return launch_route(m, x, T, idx, w, 0, (cudaStream_t)stream);
 }
 

@@ -1508,7 +1508,12 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         // P2: x records (async, overlapping the selection), selection, union
         for (int i = tid; i < T * rbH / 16; i += 256) cp_async16(acts + 16 * i, fa.xrec + 16 * i);
         const bool pub = blockIdx.x == 0;
-        for (int t = 0; t < T; ++t) {
+        if (k == 0) {  // a dense layer: no selection; the x records, then barrier 4
+            cp_async_wait_all();
+            __syncwarp();
+            asm volatile("bar.arrive 4, %0;" ::"r"(32 * (PIPE_CONSUMERS + 1)) : "memory");
+        }
+        for (int t = 0; t < T && k > 0; ++t) {
             sm.w_smem = w_s + t * k;
             // the first token's scores loaded: release the producer (barrier 4)
             cta_select_token<SyncConsumers>(fa.ws.c + (int64_t)t * E, fa.ws.s + (int64_t)t * E, E,

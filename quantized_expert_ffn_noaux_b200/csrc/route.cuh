@@ -318,6 +318,7 @@ __device__ void cta_select_token(const double *c_row, const double *s_row, int E
                                  int k, float rsf, const SelectSmem &sm, int32_t *idx_out,
                                  float *w_out, int *idx_smem = nullptr, int arrive_bar = 0,
                                  int arrive_count = 0) {
+    if (k <= 0 || E <= 0) return;  // a dense layer: nothing to select
     if (select_warp_shape(E, G, gk, k)) {
         cta_select_token_warps<Sync>(c_row, s_row, E, G, gk, k, rsf, sm, idx_out, w_out, idx_smem,
                                      arrive_bar, arrive_count);

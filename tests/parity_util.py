@@ -166,20 +166,24 @@ def compare_forward(gl, x_dev, tokens=None, check_h=True):
     out = out.cpu().numpy()[tokens]
     idx, w = idx.cpu().numpy()[tokens], w.cpu().numpy()[tokens]
     hq, hd = hq.cpu().numpy()[tokens], hd.cpu().numpy()[tokens]
-    # the oracle routes the sampled tokens itself
-    probe = oracle.Layer(synth.layer_cfg(gl.cfg), gl.Wr.cpu().numpy(), gl.bias.cpu().numpy(),
-                         [None] * (gl.cfg["n_routed"] + gl.cfg["n_shared"]))
-    ref_route = probe.route(x_host)
-    loose = check_route(idx, w, ref_route, G=gl.cfg["n_group"], gk=gl.cfg["topk_group"],
-                        rsf=gl.cfg["routed_scaling_factor"])
-    need = set(idx.reshape(-1).tolist()) | set(ref_route["idx"].reshape(-1).tolist())
-    layer = gl.oracle_layer(need)
-    # undecidable tokens: the oracle re-runs with the CUDA side's choice, which
-    # check_route has confirmed to be a valid tie alternative
-    idx_in = ref_route["idx"].copy()
-    for i in loose:
-        idx_in[i] = idx[i]
-    ref = layer.forward(x_host, idx_in=idx_in, nthreads=oracle.n_threads_default())
+    if gl.cfg["n_routed"] == 0:  # a dense layer: no routing to compare
+        layer = gl.oracle_layer(set())
+        ref = layer.forward(x_host, nthreads=oracle.n_threads_default())
+    else:
+        # the oracle routes the sampled tokens itself
+        probe = oracle.Layer(synth.layer_cfg(gl.cfg), gl.Wr.cpu().numpy(), gl.bias.cpu().numpy(),
+                             [None] * (gl.cfg["n_routed"] + gl.cfg["n_shared"]))
+        ref_route = probe.route(x_host)
+        loose = check_route(idx, w, ref_route, G=gl.cfg["n_group"], gk=gl.cfg["topk_group"],
+                            rsf=gl.cfg["routed_scaling_factor"])
+        need = set(idx.reshape(-1).tolist()) | set(ref_route["idx"].reshape(-1).tolist())
+        layer = gl.oracle_layer(need)
+        # undecidable tokens: the oracle re-runs with the CUDA side's choice, which
+        # check_route has confirmed to be a valid tie alternative
+        idx_in = ref_route["idx"].copy()
+        for i in loose:
+            idx_in[i] = idx[i]
+        ref = layer.forward(x_host, idx_in=idx_in, nthreads=oracle.n_threads_default())
     if check_h:
         np.testing.assert_array_equal(hq, ref["hq"])
         np.testing.assert_array_equal(hd, ref["hd"])
