@@ -26,7 +26,7 @@ class _Cfg(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int), ("inter", ctypes.c_int), ("n_routed", ctypes.c_int),
                 ("n_shared", ctypes.c_int), ("top_k", ctypes.c_int), ("n_group", ctypes.c_int),
                 ("topk_group", ctypes.c_int), ("bits", ctypes.c_int),
-                ("routed_scaling_factor", ctypes.c_float)]
+                ("routed_scaling_factor", ctypes.c_float), ("expert_top_p", ctypes.c_float)]
 
 
 def lib():
@@ -45,8 +45,8 @@ def lib():
         _LIB.oracle_block_sums.restype = None
         _LIB.oracle_int_dot.argtypes = [vp, vp, ci, i64, i64, vp, vp, vp]
         _LIB.oracle_int_dot.restype = None
-        _LIB.oracle_route.argtypes = [vp, i64, i64, vp, vp, ci, ci, ci, ci, cf, vp, vp, vp, vp,
-                                      vp, vp]
+        _LIB.oracle_route.argtypes = [vp, i64, i64, vp, vp, ci, ci, ci, ci, cf, cf, vp, vp, vp, vp,
+                                      vp, vp, vp]
         _LIB.oracle_route.restype = ci
         _LIB.oracle_fp8_e4m3.argtypes = [ctypes.c_uint8]
         _LIB.oracle_fp8_e4m3.restype = cf
@@ -131,8 +131,9 @@ def int_dot(codes, scales, bits, K, xq, xd):
     return out
 
 
-def route(x, Wr, bias, top_k, n_group, topk_group, rsf):
-    """Route tokens -> dict(idx, w, s, c, kmargin, gmargin)."""
+def route(x, Wr, bias, top_k, n_group, topk_group, rsf, top_p=0.0):
+    """Route tokens -> dict(idx, w, s, c, kmargin, gmargin, pmargin).  top_p in
+    (0, 1): adaptive expert top-p (dropped slots idx -1, w 0)."""
     x = _c(x, np.float32)
     if x.ndim == 1:
         x = x[None]
@@ -146,12 +147,14 @@ def route(x, Wr, bias, top_k, n_group, topk_group, rsf):
     c = np.empty((T, E), np.float64)
     km = np.empty(T, np.float64)
     gm = np.empty(T, np.float64)
+    pm = np.empty(T, np.float64)
     rc = lib().oracle_route(_p(x), T, H, _p(Wr), _p(bias), E, n_group, topk_group, top_k,
-                            float(rsf), _p(idx), _p(w), _p(s), _p(c), _p(km), _p(gm))
+                            float(rsf), float(top_p), _p(idx), _p(w), _p(s), _p(c), _p(km),
+                            _p(gm), _p(pm))
     if rc != 0:
         raise ValueError("oracle_route rejected E=%d G=%d gk=%d k=%d" % (E, n_group, topk_group,
                                                                         top_k))
-    return dict(idx=idx, w=w, s=s, c=c, kmargin=km, gmargin=gm)
+    return dict(idx=idx, w=w, s=s, c=c, kmargin=km, gmargin=gm, pmargin=pm)
 
 
 def fp8_e4m3(code):
@@ -248,12 +251,13 @@ class Layer:
     def _ccfg(self):
         c = self.cfg
         return _Cfg(c["hidden"], c["inter"], c["n_routed"], c["n_shared"], c["top_k"],
-                    c["n_group"], c["topk_group"], c["bits"], c["routed_scaling_factor"])
+                    c["n_group"], c["topk_group"], c["bits"], c["routed_scaling_factor"],
+                    c.get("expert_top_p", 0.0))
 
     def route(self, x):
         c = self.cfg
         return route(x, self.Wr, self.bias, c["top_k"], c["n_group"], c["topk_group"],
-                     c["routed_scaling_factor"])
+                     c["routed_scaling_factor"], c.get("expert_top_p", 0.0))
 
     def forward(self, x, idx_in=None, hq_in=None, hd_in=None, nthreads=1):
         """-> dict(out [T][H], idx, w, hq [T][k+S][I], hd [T][k+S][I/32])."""

@@ -257,6 +257,7 @@ void oracle_int_dot(const uint8_t *codes, const float *scales, int bits, int64_t
 typedef struct {
     int hidden, inter, n_routed, n_shared, top_k, n_group, topk_group, bits;
     float routed_scaling_factor;
+    float expert_top_p;  /* adaptive expert top-p; 0 or >= 1: off */
 } oracle_cfg;
 
 static int route_params_ok(int E, int G, int gk, int k)
@@ -329,6 +330,65 @@ static void select_token(const double *s, const double *c, int E, int G, int gk,
     for (int j = 0; j < k; ++j) w[j] = (float)((s[idx[j]] / ssum) * (double)rsf);
 }
 
+/* Adaptive expert top-p.  [HN] モデルのダウンロードと実行, useful-options
+ * bullet: --topp 0.7 "adaptive expert top-p" (30-40 % less disk traffic);
+ * the pages give no rule.  Reading: after the group-limited top-k, take the
+ * k selected experts by descending sigmoid score s (ties: the earlier slot)
+ * and keep each while the scores kept so far sum to less than p times the
+ * sum over all k (the first is always kept), so the kept experts carry at
+ * least p of the renormalised weight; the others are dropped (idx -1, w 0)
+ * and the weights are renormalised over the kept ones:
+ *   w_j = (s_j / sum_kept s) * routed_scaling_factor, sums in slot order.
+ * pmargin: the smallest |sum_before - p * sum_all| / sum_all over the
+ * decisions taken after the first (+inf if k == 1). */
+static void apply_top_p(const double *s, int k, double p, float rsf, int32_t *idx, float *w,
+                        double *pmargin)
+{
+    int order[32];
+    unsigned char kept[32];
+    double total = 0.0;
+    for (int j = 0; j < k; ++j) {
+        total += s[idx[j]];
+        order[j] = j;
+        kept[j] = 0;
+    }
+    /* slots by descending s, the earlier slot first on ties (insertion sort) */
+    for (int a = 1; a < k; ++a) {
+        int j = order[a], b = a;
+        while (b > 0 && s[idx[order[b - 1]]] < s[idx[j]]) {
+            order[b] = order[b - 1];
+            --b;
+        }
+        order[b] = j;
+    }
+    const double cut = p * total;
+    double cum = 0.0, margin = INFINITY;
+    for (int n = 0; n < k; ++n) {
+        const int j = order[n];
+        if (n > 0) {
+            const double dist = fabs(cum - cut) / total;
+            if (dist < margin) margin = dist;
+            if (!(cum < cut)) break;
+        }
+        kept[j] = 1;
+        cum += s[idx[j]];
+    }
+    double ksum = 0.0;
+    for (int j = 0; j < k; ++j)
+        if (kept[j]) ksum += s[idx[j]];
+    for (int j = 0; j < k; ++j) {
+        if (kept[j]) {
+            w[j] = (float)((s[idx[j]] / total) * (double)rsf);
+        } else {
+            idx[j] = -1;
+            w[j] = 0.0f;
+        }
+    }
+    if (pmargin) *pmargin = margin;
+}
+
+static int top_p_on(float p) { return p > 0.0f && p < 1.0f; }
+
 static void token_scores(const float *xt, int64_t H, const float *Wr, const float *bias, int E,
                          double *s, double *c)
 {
@@ -342,10 +402,12 @@ static void token_scores(const float *xt, int64_t H, const float *Wr, const floa
 }
 
 /* Route T tokens.  Optional outputs (may be NULL): s_out/c_out [T][E],
- * kmargin/gmargin [T].  Returns 0, or -1 on invalid parameters. */
+ * kmargin/gmargin/pmargin [T].  top_p in (0, 1) applies the adaptive expert
+ * top-p (dropped slots: idx -1, w 0).  Returns 0, or -1 on invalid parameters. */
 int oracle_route(const float *x, int64_t T, int64_t H, const float *Wr, const float *bias,
-                 int E, int G, int gk, int k, float rsf, int32_t *idx, float *w,
-                 double *s_out, double *c_out, double *kmargin, double *gmargin)
+                 int E, int G, int gk, int k, float rsf, float top_p, int32_t *idx, float *w,
+                 double *s_out, double *c_out, double *kmargin, double *gmargin,
+                 double *pmargin)
 {
     if (!route_params_ok(E, G, gk, k)) return -1;
     double *s = malloc(sizeof(double) * E), *c = malloc(sizeof(double) * E);
@@ -355,6 +417,9 @@ int oracle_route(const float *x, int64_t T, int64_t H, const float *Wr, const fl
         token_scores(x + t * H, H, Wr, bias, E, s, c);
         double km, gm;
         select_token(s, c, E, G, gk, k, rsf, idx + t * k, w + t * k, &km, &gm, gs, gkeep, taken);
+        double pm = INFINITY;
+        if (top_p_on(top_p)) apply_top_p(s, k, (double)top_p, rsf, idx + t * k, w + t * k, &pm);
+        if (pmargin) pmargin[t] = pm;
         if (s_out) memcpy(s_out + t * E, s, sizeof(double) * E);
         if (c_out) memcpy(c_out + t * E, c, sizeof(double) * E);
         if (kmargin) kmargin[t] = km;
@@ -482,15 +547,19 @@ int oracle_moe_forward(const oracle_cfg *cfg, const float *Wr, const float *bias
             double km, gm;
             select_token(s, c, E, G, gk, k, cfg->routed_scaling_factor, idx + t * k, w + t * k,
                          &km, &gm, gs, gkeep, taken);
-            if (idx_in) {
+            if (top_p_on(cfg->expert_top_p))
+                apply_top_p(s, k, (double)cfg->expert_top_p, cfg->routed_scaling_factor,
+                            idx + t * k, w + t * k, NULL);
+            if (idx_in) {  /* another side's choice; -1 marks a dropped slot */
                 double ssum = 0.0;
                 for (int j = 0; j < k; ++j) {
                     idx[t * k + j] = idx_in[t * k + j];
-                    ssum += s[idx_in[t * k + j]];
+                    if (idx_in[t * k + j] >= 0) ssum += s[idx_in[t * k + j]];
                 }
                 for (int j = 0; j < k; ++j)
-                    w[t * k + j] = (float)((s[idx_in[t * k + j]] / ssum) *
-                                           (double)cfg->routed_scaling_factor);
+                    w[t * k + j] = idx_in[t * k + j] < 0 ? 0.0f
+                                   : (float)((s[idx_in[t * k + j]] / ssum) *
+                                             (double)cfg->routed_scaling_factor);
             }
         }
         free(s); free(c); free(gs); free(gkeep); free(taken);
@@ -503,6 +572,7 @@ int oracle_moe_forward(const oracle_cfg *cfg, const float *Wr, const float *bias
     for (int64_t t = 0; t < T && !missing; ++t)
         for (int j = 0; j < slots; ++j) {
             int e = j < k ? idx[t * k + j] : E + (j - k);
+            if (j < k && e == -1) continue;  /* a slot top-p dropped */
             if (e < 0 || e >= E + S) { missing = 1; break; }
             for (int m = 0; m < 3; ++m)
                 if (!mats[e * 3 + m].codes || !mats[e * 3 + m].scales) missing = 1;
@@ -522,8 +592,15 @@ int oracle_moe_forward(const oracle_cfg *cfg, const float *Wr, const float *bias
             /* shared experts first, then routed slots in order */
             int j = jj < S ? k + jj : jj - S;
             int ex = j < k ? idx[t * k + j] : E + (j - k);
-            const oracle_qmat *m3 = mats + (int64_t)ex * 3;
             int64_t hs = (t * slots + j);
+            if (ex < 0) {  /* a slot top-p dropped: no expert, no contribution */
+                if (hq_out) memset(hq_out + hs * I, 0, (size_t)I);
+                if (hd_out) memset(hd_out + hs * (I / QBLK), 0, sizeof(float) * (size_t)(I / QBLK));
+                if (jj == 0)
+                    for (int64_t r = 0; r < H; ++r) acc[r] = 0.0;
+                continue;
+            }
+            const oracle_qmat *m3 = mats + (int64_t)ex * 3;
             const int8_t *hqi = hq_in ? hq_in + hs * I : NULL;
             const float *hdi = hd_in ? hd_in + hs * (I / QBLK) : NULL;
             int8_t *hqo = hq_out ? hq_out + hs * I : hq_tmp;

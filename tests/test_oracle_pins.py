@@ -244,6 +244,95 @@ def test_route_matches_brute_force(E, G, gk, k):
         assert abs(float(r["w"][0].astype(np.float64).sum()) - 2.5) < 1e-5
 
 
+@pytest.mark.parametrize("E,G,gk,k", [(8, 1, 1, 4), (16, 4, 2, 5), (12, 3, 2, 6)])
+@pytest.mark.parametrize("p", [0.3, 0.5, 0.7, 0.9])
+def test_top_p_keeps_a_smallest_subset_reaching_p(E, G, gk, k, p):
+    """Adaptive expert top-p, checked by brute force over subsets: the kept
+    experts are a smallest subset of the top-k whose scores reach p of the
+    top-k's score sum, they are the largest scores, at least one is kept,
+    dropped slots read -1 / 0, and the weights renormalise over the kept."""
+    H = 64
+    for trial in range(10):
+        x = RNG.standard_normal(H).astype(np.float32)
+        Wr = (RNG.standard_normal((E, H)) / 8.0).astype(np.float32)
+        b = RNG.uniform(-0.1, 0.1, E).astype(np.float32)
+        full = oracle.route(x, Wr, b, k, G, gk, 2.5)
+        r = oracle.route(x, Wr, b, k, G, gk, 2.5, top_p=p)
+        s, c = _exact_scores(x, Wr, b)
+        sel = full["idx"][0].tolist()
+        kept = [e for e in r["idx"][0].tolist() if e >= 0]
+        assert set(kept) <= set(sel) and len(kept) >= 1
+        for j, e in enumerate(r["idx"][0].tolist()):       # slots keep their places
+            assert e == -1 or e == sel[j]
+        if r["pmargin"][0] < 1e-9:
+            continue                                       # a cut on the boundary itself
+        total = sum(s[e] for e in sel)
+        m = min(n for n in range(1, k + 1)
+                if any(sum(s[e] for e in sub) >= p * total
+                       for sub in itertools.combinations(sel, n)))
+        assert len(kept) == m
+        top = sorted(sel, key=lambda e: -s[e])[:m]
+        assert sorted(kept) == sorted(top)
+        w = r["w"][0]
+        assert np.all(w[r["idx"][0] < 0] == 0)
+        ks = np.array([s[e] for e in kept])
+        np.testing.assert_allclose(w[r["idx"][0] >= 0], ks / ks.sum() * 2.5, rtol=1e-6)
+
+
+def test_top_p_off_values_and_one_kept():
+    E, H, k = 16, 64, 4
+    x = RNG.standard_normal((6, H)).astype(np.float32)
+    Wr = (RNG.standard_normal((E, H)) / 8.0).astype(np.float32)
+    b = RNG.uniform(-0.1, 0.1, E).astype(np.float32)
+    base = oracle.route(x, Wr, b, k, 4, 2, 2.5)
+    for off in (0.0, 1.0, 1.5):
+        r = oracle.route(x, Wr, b, k, 4, 2, 2.5, top_p=off)
+        np.testing.assert_array_equal(r["idx"], base["idx"])
+        np.testing.assert_array_equal(r["w"], base["w"])
+    r = oracle.route(x, Wr, b, k, 4, 2, 2.5, top_p=1e-6)   # only the largest s survives
+    for t in range(6):
+        kept = r["idx"][t][r["idx"][t] >= 0]
+        assert len(kept) == 1
+        assert kept[0] == max(base["idx"][t], key=lambda e: base["s"][t][e])
+        assert r["w"][t][r["idx"][t] >= 0][0] == np.float32(2.5)
+
+
+def test_top_p_exact_boundary_and_ties():
+    """Zero router weights make every score exactly 0.5 (the bias alone
+    orders the choice): with k = 4 and p = 1/2 the first two slots reach
+    exactly half the sum, so the cut falls after them -- reaching p stops the
+    keeping -- and equal scores keep the earlier slots."""
+    E, H, k = 8, 32, 4
+    x = RNG.standard_normal((1, H)).astype(np.float32)
+    Wr = np.zeros((E, H), np.float32)
+    b = np.array([0.01, 0.05, 0.02, 0.07, 0.03, 0.0, 0.06, 0.04], np.float32)
+    r = oracle.route(x, Wr, b, k, 1, 1, 2.0, top_p=0.5)
+    assert r["idx"][0].tolist() == [3, 6, -1, -1]   # slots by c: 3, 6, 1, 7
+    np.testing.assert_array_equal(r["w"][0], np.array([1.0, 1.0, 0.0, 0.0], np.float32))
+    r = oracle.route(x, Wr, b, k, 1, 1, 2.0, top_p=0.75)
+    assert r["idx"][0].tolist() == [3, 6, 1, -1]
+
+
+def test_top_p_layer_with_one_kept_expert():
+    """With a single kept expert the layer is e_shared + rsf * e_kept exactly
+    (its renormalised weight is rsf: s / s = 1)."""
+    rng = np.random.default_rng(31)
+    cfg = _cfg(n_routed=8, top_k=3, n_group=4, topk_group=2, expert_top_p=1e-6)
+    layer = _layer(cfg, rng)
+    x = rng.standard_normal((4, 64)).astype(np.float32)
+    res = layer.forward(x)
+    xq, xd = oracle.quant_q8(x)
+    for t in range(4):
+        kept = res["idx"][t][res["idx"][t] >= 0]
+        assert len(kept) == 1 and res["w"][t][res["idx"][t] >= 0][0] == np.float32(2.5)
+        e_sh = oracle.expert(64, 32, 4, layer.experts[-1], xq[t], xd[t])[0].astype(np.float64)
+        e_k = oracle.expert(64, 32, 4, layer.experts[kept[0]], xq[t], xd[t])[0].astype(np.float64)
+        np.testing.assert_array_equal(res["out"][t], (e_sh + 2.5 * e_k).astype(np.float32))
+        # dropped slots carry no intermediate
+        for j in np.nonzero(res["idx"][t] < 0)[0]:
+            assert np.all(res["hq"][t, j] == 0) and np.all(res["hd"][t, j] == 0)
+
+
 def test_route_bias_shift_invariance_and_plain_topk():
     E, H, k = 32, 64, 6
     x = RNG.standard_normal((5, H)).astype(np.float32)
