@@ -378,7 +378,7 @@ static void apply_top_p(const double *s, int k, double p, float rsf, int32_t *id
         if (kept[j]) ksum += s[idx[j]];
     for (int j = 0; j < k; ++j) {
         if (kept[j]) {
-            w[j] = (float)((s[idx[j]] / total) * (double)rsf);
+            w[j] = (float)((s[idx[j]] / ksum) * (double)rsf);
         } else {
             idx[j] = -1;
             w[j] = 0.0f;
