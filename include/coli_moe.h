@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-#define COLI_ABI_VERSION 1
+#define COLI_ABI_VERSION 2
 
 /* A cudaStream_t, declared without the CUDA headers. */
 typedef struct CUstream_st *coli_stream_t;
@@ -77,12 +77,23 @@ typedef enum { COLI_W_INT8 = 8, COLI_W_INT4 = 4, COLI_W_INT2 = 2 } coli_wfmt;
  *   n_routed (E) in [1, 1024], n_shared (S) in [0, 4].
  *   n_group (G) divides E; topk_group (gk) in [1, G];
  *   top_k (k) in [1, min(32, gk*E/G)].
- *   max_tokens: largest T any call on this handle will pass, >= 1. */
+ *   A dense layer ([HN] router bullet: the first three layers are dense) is
+ *   E = 0 with k = 0 and S >= 1 (G and gk ignored): every token through the
+ *   shared experts only; its router pointers may be NULL.
+ *   max_tokens: largest T any call on this handle will pass, >= 1.
+ *   expert_top_p: adaptive expert top-p ([HN] モデルのダウンロードと実行,
+ *     --topp; 0 or >= 1: off).  For p in (0, 1), after the group-limited
+ *     top-k the selected experts are kept by descending sigmoid score (ties:
+ *     the earlier slot) while the kept scores sum to less than p times the
+ *     top-k's score sum, the first always; the other slots are dropped
+ *     (idx -1, weight 0, no expert computed) and the weights renormalised
+ *     over the kept experts. */
 typedef struct {
     int hidden, inter, n_routed, n_shared, top_k, n_group, topk_group;
     float routed_scaling_factor;
     int wfmt; /* a coli_wfmt */
     int max_tokens;
+    float expert_top_p;
 } coli_moe_config;
 
 /* One quantised matrix: codes [rows][K*bits/8] bytes, row-major with K
@@ -145,7 +156,8 @@ coli_status coli_moe_create(const coli_moe_config *cfg, const float *router_w, c
 
 /* Routing only ([HN] router bullet):  x [T][H] fp32 ->
  *   idx [T][k] int32: selected experts sorted by descending choice score
- *                     c = sigmoid(x.W_r) + bias (ties: lower index);
+ *                     c = sigmoid(x.W_r) + bias (ties: lower index); -1 for a
+ *                     slot the adaptive expert top-p dropped;
  *   w   [T][k] fp32:  sigmoid scores of idx renormalised to sum 1, times
  *                     routed_scaling_factor (the bias is not in w).
  * Group-limited: a group's score is the sum of its two best c; only the

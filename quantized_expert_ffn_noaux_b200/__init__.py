@@ -42,7 +42,8 @@ class _Config(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int), ("inter", ctypes.c_int), ("n_routed", ctypes.c_int),
                 ("n_shared", ctypes.c_int), ("top_k", ctypes.c_int), ("n_group", ctypes.c_int),
                 ("topk_group", ctypes.c_int), ("routed_scaling_factor", ctypes.c_float),
-                ("wfmt", ctypes.c_int), ("max_tokens", ctypes.c_int)]
+                ("wfmt", ctypes.c_int), ("max_tokens", ctypes.c_int),
+                ("expert_top_p", ctypes.c_float)]
 
 
 class _KTime(ctypes.Structure):
@@ -166,7 +167,8 @@ def dbg_block_sums(codes, bits, K, xq, stream=None):
 def _config(cfg, max_tokens=None):
     return _Config(cfg["hidden"], cfg["inter"], cfg["n_routed"], cfg["n_shared"], cfg["top_k"],
                    cfg["n_group"], cfg["topk_group"], cfg["routed_scaling_factor"], cfg["bits"],
-                   cfg.get("max_tokens", 1) if max_tokens is None else max_tokens)
+                   cfg.get("max_tokens", 1) if max_tokens is None else max_tokens,
+                   cfg.get("expert_top_p", 0.0))
 
 
 def router_static(cfg, router_w, bias, x, idx=None, w=None, stream=None):
@@ -214,7 +216,7 @@ class MoELayer:
         self._keep = (router_w, bias, list(experts))
         c = _Config(cfg["hidden"], cfg["inter"], cfg["n_routed"], cfg["n_shared"], cfg["top_k"],
                     cfg["n_group"], cfg["topk_group"], cfg["routed_scaling_factor"], cfg["bits"],
-                    cfg["max_tokens"])
+                    cfg["max_tokens"], cfg.get("expert_top_p", 0.0))
         arr = (_Expert * len(experts))()
         for i, ex in enumerate(experts):
             arr[i] = _Expert(*(_QMat(m[0].data_ptr(), m[1].data_ptr())
@@ -238,9 +240,7 @@ class MoELayer:
 
     def workspace_bytes(self):
         c = self.cfg
-        cc = _Config(c["hidden"], c["inter"], c["n_routed"], c["n_shared"], c["top_k"],
-                     c["n_group"], c["topk_group"], c["routed_scaling_factor"], c["bits"],
-                     c["max_tokens"])
+        cc = _config(c)
         return int(lib().coli_moe_workspace_bytes(ctypes.byref(cc)))
 
     def router(self, x, idx=None, w=None, stream=None):

@@ -163,6 +163,7 @@ bool cfg_valid(const coli_moe_config *c, std::string *why) {
     if (c->top_k < 1 || c->top_k > 32 || c->top_k > cand)
         return bad("top_k must be in [1, min(32, topk_group * n_routed / n_group)]");
     if (!(c->routed_scaling_factor == c->routed_scaling_factor)) return bad("routed_scaling_factor is NaN");
+    if (!(c->expert_top_p == c->expert_top_p)) return bad("expert_top_p is NaN");
     if (c->max_tokens < 1 || c->max_tokens > (1 << 20)) return bad("max_tokens must be in [1, 2^20]");
     return true;
 }
@@ -495,7 +496,7 @@ coli_status launch_route(coli_moe *m, const float *x, int T, int32_t *idx, float
         const size_t smem = select_smem(c) + 4 * (size_t)c.n_routed + 4 * (size_t)T * c.top_k;
         int occ = 1;
         void (*kern)(const float *, int, int, const float *, const float *, int, int, int, int,
-                     int, float, RouteWs, uint8_t *, int8_t *, float *, int, int32_t *, float *);
+                     int, float, RouteWs, uint8_t *, int8_t *, float *, int, int32_t *, float *, float);
         if (T <= 1) kern = k_router_small<1, 4>;
         else if (T <= 2) kern = k_router_small<2, 4>;
         else if (T <= 4) kern = k_router_small<4, 4>;
@@ -505,7 +506,7 @@ coli_status launch_route(coli_moe *m, const float *x, int T, int32_t *idx, float
         Launch L(m, s, "router");
         kern<<<E, 256, smem, s>>>(x, T, H, m->router_w, m->bias, E, c.n_shared, c.n_group,
                                   c.topk_group, c.top_k, c.routed_scaling_factor, m->rw, nullptr,
-                                  nullptr, nullptr, 0, idx, w);
+                                  nullptr, nullptr, 0, idx, w, c.expert_top_p);
         return L.done();
     }
     if (E > 0) {
@@ -535,7 +536,8 @@ coli_status launch_route(coli_moe *m, const float *x, int T, int32_t *idx, float
         if (st != COLI_OK) return st;
         Launch L(m, s, "router_select");
         k_route_select<<<T, 256, smem, s>>>(m->rw, T, E, c.n_shared, c.n_group, c.topk_group,
-                                            c.top_k, c.routed_scaling_factor, idx, w, do_union);
+                                            c.top_k, c.routed_scaling_factor, idx, w, do_union,
+                                            c.expert_top_p);
         return L.done();
     }
 }
@@ -562,6 +564,7 @@ coli_status launch_small_path(coli_moe *m, const float *x, int T, float *out, cu
     fa.gk = c.topk_group;
     fa.k = c.top_k;
     fa.rsf = c.routed_scaling_factor;
+    fa.top_p = c.expert_top_p;
     fa.ws = m->rw;
     fa.experts = m->experts_dev;
     fa.xrec = m->xrec;
@@ -1208,6 +1211,7 @@ coli_status coli_router_static(const coli_moe_config *cfg, const float *router_w
     g_last_error.clear();
     std::string why;
     if (!cfg_valid(cfg, &why)) return fail(COLI_EINVAL, "invalid config: %s", why.c_str());
+    if (cfg->n_routed == 0) return fail(COLI_EINVAL, "a dense layer has no router");
     if (T < 1 || T > ROUTER_STATIC_MAX_T)
         return fail(COLI_EINVAL, "coli_router_static takes 1 <= T <= %d tokens (got %d)",
                     ROUTER_STATIC_MAX_T, T);
@@ -1232,7 +1236,7 @@ coli_status coli_router_static(const coli_moe_config *cfg, const float *router_w
     COLI_CUDA(cudaMemsetAsync(rw.counter, 0, sizeof(uint32_t), s), "clear router ticket");
     const size_t smem = select_smem(*cfg) + 4 * (size_t)E + 4 * (size_t)T * cfg->top_k;
     void (*kern)(const float *, int, int, const float *, const float *, int, int, int, int, int,
-                 float, RouteWs, uint8_t *, int8_t *, float *, int, int32_t *, float *);
+                 float, RouteWs, uint8_t *, int8_t *, float *, int, int32_t *, float *, float);
     if (T <= 1) kern = k_router_small<1, 4>;
     else if (T <= 2) kern = k_router_small<2, 4>;
     else if (T <= 4) kern = k_router_small<4, 4>;
@@ -1242,7 +1246,7 @@ coli_status coli_router_static(const coli_moe_config *cfg, const float *router_w
     Launch L(nullptr, s, "router_static");
     kern<<<E, 256, smem, s>>>(x, T, cfg->hidden, router_w, bias, E, cfg->n_shared, cfg->n_group,
                               cfg->topk_group, cfg->top_k, cfg->routed_scaling_factor, rw, nullptr,
-                              nullptr, nullptr, 0, idx, w);
+                              nullptr, nullptr, 0, idx, w, cfg->expert_top_p);
     return L.done();
 }
 

@@ -851,6 +851,7 @@ struct DecodeArgs {
     const float *bias;
     int T, H, I, E, S, G, gk, k;
     float rsf;
+    float top_p;        // adaptive expert top-p (0 or >= 1: off)
     RouteWs ws;
     const ExpertDev *experts;
     uint8_t *xrec;
@@ -1519,7 +1520,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
             cta_select_token<SyncConsumers>(fa.ws.c + (int64_t)t * E, fa.ws.s + (int64_t)t * E, E,
                                             fa.G, fa.gk, k, fa.rsf, sm, pub ? fa.ws.idx + t * k : nullptr,
                                             pub ? fa.ws.w + t * k : nullptr, idx_s + t * k, 4,
-                                            t == 0 ? 32 * (PIPE_CONSUMERS + 1) : 0);
+                                            t == 0 ? 32 * (PIPE_CONSUMERS + 1) : 0, fa.top_p);
         }
         if (MAXT == 1) {
             if (warp == 0) warp_union_one(lw, E, S, k, idx_s);
@@ -1536,8 +1537,9 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
             for (int i = tid; i < np; i += 256) {
                 fa.ws.pair_tok[i] = lw.pair_tok[i];
                 fa.ws.pair_slot[i] = lw.pair_slot[i];
-                fa.ws.tok_pair[i] = lw.tok_pair[i];
             }
+            // one entry per (token, slot): more than np where slots hold -1
+            for (int i = tid; i < T * (k + S); i += 256) fa.ws.tok_pair[i] = lw.tok_pair[i];
             if (tid == 0) *fa.ws.n_active = na;
         }
     }

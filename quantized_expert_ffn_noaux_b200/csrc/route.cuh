@@ -212,6 +212,51 @@ __device__ inline SelectSmem carve_select(void *base, int E, int G) {
     return m;
 }
 
+// Adaptive expert top-p of one token, by one warp after the top-k
+// ("Show HN: 遅いコンピュータで GLM 5.2 を実行する", モデルのダウンロードと実行,
+// --topp; reading: keep the selected experts by descending sigmoid score,
+// ties to the earlier slot, while the kept scores sum to less than
+// p * (sum over the k), the first always; drop the rest; renormalise over the
+// kept).  Lane j < k holds slot j's expert ej and score sj; slot_s[0..k) holds
+// the same scores in slot order and `total` their slot-order sum.  On return
+// ej is -1 for a dropped slot and the result is the slot's weight.  order /
+// kept: shared scratch of k ints each.  Every operation on the scores is the
+// definition's, in its order (one lane runs the cumulative sum).
+__device__ __forceinline__ float warp_top_p(int &ej, double sj, const double *slot_s, int k,
+                                            double total, float p, float rsf, int *order,
+                                            int *kept) {
+    const int lane = threadIdx.x & 31;
+    if (lane < k) {
+        int r = 0;
+        for (int i = 0; i < k; ++i) {
+            const double u = slot_s[i];
+            r += (int)(u > sj) | ((int)(u == sj) & (int)(i < lane));
+        }
+        order[r] = lane;
+        kept[lane] = 0;
+    }
+    __syncwarp();
+    if (lane == 0) {
+        const double cut = (double)p * total;
+        double cum = 0.0;
+        for (int n = 0; n < k; ++n) {
+            const int j = order[n];
+            if (n > 0 && !(cum < cut)) break;
+            kept[j] = 1;
+            cum += slot_s[j];
+        }
+    }
+    __syncwarp();
+    double ksum = 0.0;
+    for (int i = 0; i < k; ++i)
+        if (kept[i]) ksum += slot_s[i];
+    const bool keep = lane < k && kept[lane];
+    if (!keep) ej = -1;
+    return keep ? (float)((sj / ksum) * (double)rsf) : 0.0f;
+}
+
+__host__ __device__ inline bool top_p_on(float p) { return p > 0.0f && p < 1.0f; }
+
 // Warp-level selection for the common shape: every group fits one warp
 // (E/G <= 32), at most 8 groups, and the kept groups' candidates fit one warp
 // (topk_group * min(top_k, E/G) <= 32).  Warp g holds group g, one expert per
@@ -226,7 +271,7 @@ template <typename Sync>
 __device__ void cta_select_token_warps(const double *c_row, const double *s_row, int E, int G,
                                        int gk, int k, float rsf, const SelectSmem &sm,
                                        int32_t *idx_out, float *w_out, int *idx_smem,
-                                       int arrive_bar, int arrive_count) {
+                                       int arrive_bar, int arrive_count, float top_p) {
     const unsigned FULL = 0xffffffffu;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int per = E / G, kk = k < per ? k : per;
@@ -297,9 +342,12 @@ __device__ void cta_select_token_warps(const double *c_row, const double *s_row,
         double ssum = 0.0;
 #pragma unroll 8
         for (int j = 0; j < k; ++j) ssum += sm.c[j];
+        int ej = lane < k ? sm.sel[lane] : 0;
+        float wj = lane < k ? (float)((sm.c[lane] / ssum) * (double)rsf) : 0.0f;
+        if (top_p_on(top_p))
+            wj = warp_top_p(ej, lane < k ? sm.c[lane] : 0.0, sm.c, k, ssum, top_p, rsf, sm.cand,
+                            sm.grank);
         if (lane < k) {
-            const int ej = sm.sel[lane];
-            const float wj = (float)((sm.c[lane] / ssum) * (double)rsf);
             if (idx_out) idx_out[lane] = ej;
             if (w_out) w_out[lane] = wj;
             if (idx_smem) idx_smem[lane] = ej;
@@ -317,11 +365,11 @@ template <typename Sync = SyncAll>
 __device__ void cta_select_token(const double *c_row, const double *s_row, int E, int G, int gk,
                                  int k, float rsf, const SelectSmem &sm, int32_t *idx_out,
                                  float *w_out, int *idx_smem = nullptr, int arrive_bar = 0,
-                                 int arrive_count = 0) {
+                                 int arrive_count = 0, float top_p = 0.0f) {
     if (k <= 0 || E <= 0) return;  // a dense layer: nothing to select
     if (select_warp_shape(E, G, gk, k)) {
         cta_select_token_warps<Sync>(c_row, s_row, E, G, gk, k, rsf, sm, idx_out, w_out, idx_smem,
-                                     arrive_bar, arrive_count);
+                                     arrive_bar, arrive_count, top_p);
         return;
     }
     const int tid = threadIdx.x, nthr = 256;
@@ -414,11 +462,17 @@ __device__ void cta_select_token(const double *c_row, const double *s_row, int E
             const double v = __shfl_sync(0xffffffffu, sj, j);
             if (j < k) ssum += v;
         }
+        int ej = e;
+        float wj = lane < k ? (float)((sj / ssum) * (double)rsf) : 0.0f;
+        if (top_p_on(top_p)) {
+            if (lane < k) sm.candc[lane] = sj;  // slot-order scores (candc is free by now)
+            __syncwarp();
+            wj = warp_top_p(ej, sj, sm.candc, k, ssum, top_p, rsf, sm.cand, sm.grank);
+        }
         if (lane < k) {
-            const float wj = (float)((sj / ssum) * (double)rsf);
-            if (idx_out) idx_out[lane] = e;
+            if (idx_out) idx_out[lane] = ej;
             if (w_out) w_out[lane] = wj;
-            if (idx_smem) idx_smem[lane] = e;
+            if (idx_smem) idx_smem[lane] = ej;
             if (sm.w_smem) sm.w_smem[lane] = wj;
         }
     }
@@ -476,14 +530,14 @@ __device__ void warp_union_one(RouteWs ws, int E, int S, int k, const int *idx /
 // builds the batch-union tables.  Dynamic smem: select_smem_bytes(E, G).
 __global__ void __launch_bounds__(256) k_route_select(
     RouteWs ws, int T, int E, int S, int G, int gk, int k, float rsf, int32_t *__restrict__ idx_out,
-    float *__restrict__ w_out, int do_union) {
+    float *__restrict__ w_out, int do_union, float top_p) {
     extern __shared__ __align__(16) double smem_d[];
     __shared__ int is_last;
     __shared__ int scan_tmp[8];
     const int t = blockIdx.x, tid = threadIdx.x;
     const SelectSmem sm = carve_select(smem_d, E, G);
     cta_select_token(ws.c + (int64_t)t * E, ws.s + (int64_t)t * E, E, G, gk, k, rsf, sm,
-                     idx_out + (int64_t)t * k, w_out + (int64_t)t * k);
+                     idx_out + (int64_t)t * k, w_out + (int64_t)t * k, nullptr, 0, 0, top_p);
     double *c_s = sm.c;
     const int *sel = idx_out + (int64_t)t * k;
     if (!do_union) return;
@@ -656,7 +710,7 @@ __global__ void __launch_bounds__(256) k_router_small(
     const float *__restrict__ x, int T, int H, const float *__restrict__ Wr,
     const float *__restrict__ bias, int E, int S, int G, int gk, int k, float rsf, RouteWs ws,
     uint8_t *__restrict__ xrec, int8_t *__restrict__ xq, float *__restrict__ xd,
-    int do_union, int32_t *__restrict__ idx_out, float *__restrict__ w_out) {
+    int do_union, int32_t *__restrict__ idx_out, float *__restrict__ w_out, float top_p) {
     extern __shared__ __align__(16) uint8_t smem_r[];
     __shared__ double red[8][NT];
     __shared__ int is_last;
@@ -721,7 +775,7 @@ __global__ void __launch_bounds__(256) k_router_small(
     int *idx_s = cnt + E;
     for (int t = 0; t < T; ++t)
         cta_select_token(ws.c + (int64_t)t * E, ws.s + (int64_t)t * E, E, G, gk, k, rsf, sm,
-                         idx_dst + t * k, w_dst + t * k, idx_s + t * k);
+                         idx_dst + t * k, w_dst + t * k, idx_s + t * k, 0, 0, top_p);
     if (do_union) cta_union_small(ws, T, E, S, k, cnt, idx_s, scan_tmp);
     __syncthreads();
     if (tid == 0) *ws.counter = 0u;

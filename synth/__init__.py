@@ -55,7 +55,10 @@ def layer_cfg(cfg):
     """The layer-shape keys only."""
     keys = ("hidden", "inter", "n_routed", "n_shared", "top_k", "n_group", "topk_group",
             "routed_scaling_factor", "bits")
-    return {k: cfg[k] for k in keys}
+    out = {k: cfg[k] for k in keys}
+    if cfg.get("expert_top_p"):
+        out["expert_top_p"] = cfg["expert_top_p"]
+    return out
 
 
 def seed_for(*parts):

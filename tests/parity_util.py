@@ -73,7 +73,10 @@ class GpuLayer:
 
 
 def decidable(route_res, t):
-    return route_res["kmargin"][t] > MARGIN and route_res["gmargin"][t] > MARGIN
+    ok = route_res["kmargin"][t] > MARGIN and route_res["gmargin"][t] > MARGIN
+    if "pmargin" in route_res:  # the adaptive expert top-p's cut
+        ok = ok and route_res["pmargin"][t] > MARGIN
+    return ok
 
 
 def _group_scores(c, G):
@@ -126,6 +129,20 @@ def check_route(gpu_idx, gpu_w, ref, tokens=None, G=None, gk=None, rsf=None):
     for i, t in enumerate(tokens):
         gi, ri = gpu_idx[i], ref["idx"][t]
         c = ref["c"][t]
+        if (gi < 0).any() or (ri < 0).any():
+            # adaptive expert top-p dropped slots (-1, weight 0; slots keep their places)
+            kept = gi[gi >= 0]
+            assert len(set(kept.tolist())) == len(kept) and len(kept) >= 1, (t, gi)
+            assert np.all(gpu_w[i][gi < 0] == 0), (t, gi, gpu_w[i])
+            if decidable(ref, t):
+                np.testing.assert_array_equal(gi, ri)
+                np.testing.assert_allclose(gpu_w[i], ref["w"][t], rtol=1e-6)
+            else:
+                s = ref["s"][t][kept]
+                scale = float(ref["w"][t].astype(np.float64).sum()) if rsf is None else rsf
+                np.testing.assert_allclose(gpu_w[i][gi >= 0], s / s.sum() * scale, rtol=1e-6)
+                loose.append(i)
+            continue
         if not decidable(ref, t):
             assert G is not None and gk is not None, "check_route needs G, gk for near ties"
             assert valid_tie_choice(gi, c, G, gk, len(ri)), (t, gi, ri)
@@ -177,6 +194,7 @@ def compare_forward(gl, x_dev, tokens=None, check_h=True):
         loose = check_route(idx, w, ref_route, G=gl.cfg["n_group"], gk=gl.cfg["topk_group"],
                             rsf=gl.cfg["routed_scaling_factor"])
         need = set(idx.reshape(-1).tolist()) | set(ref_route["idx"].reshape(-1).tolist())
+        need.discard(-1)  # a slot the adaptive expert top-p dropped
         layer = gl.oracle_layer(need)
         # undecidable tokens: the oracle re-runs with the CUDA side's choice, which
         # check_route has confirmed to be a valid tie alternative

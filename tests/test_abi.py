@@ -36,7 +36,7 @@ def test_header_declares_the_boundary():
 def test_every_declared_symbol_is_exported(L):
     missing = [n for n in declared_functions() if not hasattr(L, n)]
     assert not missing, missing
-    assert L.coli_abi_version() == 1
+    assert L.coli_abi_version() == 2
 
 
 def test_status_strings(L):
@@ -50,13 +50,14 @@ def _cfg(**kw):
     c.update(kw)
     return qe._Config(c["hidden"], c["inter"], c["n_routed"], c["n_shared"], c["top_k"],
                       c["n_group"], c["topk_group"], c["routed_scaling_factor"], c["wfmt"],
-                      c["max_tokens"])
+                      c["max_tokens"], c.get("expert_top_p", 0.0))
 
 
 @pytest.mark.parametrize("bad", [dict(hidden=250), dict(inter=0), dict(wfmt=3),
                                  dict(n_group=3), dict(topk_group=2), dict(top_k=9),
                                  dict(top_k=0), dict(max_tokens=0), dict(n_shared=5),
-                                 dict(wfmt=2, hidden=288)])
+                                 dict(wfmt=2, hidden=288), dict(expert_top_p=float("nan")),
+                                 dict(n_routed=0, top_k=1), dict(n_routed=0, top_k=0, n_shared=0)])
 def test_invalid_configs_are_rejected_on_the_host(L, bad):
     c = _cfg(**bad)
     assert L.coli_moe_workspace_bytes(ctypes.byref(c)) == 0
