@@ -47,3 +47,58 @@ def test_router_static_rejects_sizes_beyond_its_scratch():
     with pytest.raises(qe.ColiError) as ei:
         qe.router_static(synth.layer_cfg(cfg), W, b, x)
     assert ei.value.status == qe.COLI_EINVAL and "T <=" in str(ei.value)
+
+
+def test_router_static_leaves_free_memory_unchanged():
+    """After the first call (which looks up the fixed array's address), further
+    calls with preallocated outputs take no device memory: the device's free
+    memory, as the driver reports it, is the same before and after them."""
+    cfg = synth.workload("glm52_decode_int4_t1")
+    W, b = synth.router(cfg, device=DEV)
+    x = synth.tokens(cfg, T=8, device=DEV, stream=7)
+    k = cfg["top_k"]
+    idx = torch.empty((8, k), dtype=torch.int32, device=DEV)
+    w = torch.empty((8, k), dtype=torch.float32, device=DEV)
+    lc = synth.layer_cfg(cfg)
+    qe.router_static(lc, W, b, x, idx=idx, w=w)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for T in (8, 1, 5, 8):
+        qe.router_static(lc, W, b, x[:T], idx=idx[:T], w=w[:T])
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+
+
+def test_router_static_rejects_more_experts_than_its_scratch():
+    cfg = synth.workload("glm52_decode_int4_t1", n_routed=1025, n_group=1, topk_group=1)
+    W, b = synth.router(cfg, device=DEV)
+    x = synth.tokens(cfg, T=1, device=DEV)
+    with pytest.raises(qe.ColiError) as ei:
+        qe.router_static(synth.layer_cfg(cfg), W, b, x)
+    assert ei.value.status == qe.COLI_EINVAL and "1024" in str(ei.value)
+
+
+def test_router_static_rejects_a_dense_layer():
+    cfg = synth.workload("glm52_decode_int4_t1")
+    W, b = synth.router(cfg, device=DEV)
+    x = synth.tokens(cfg, T=1, device=DEV)
+    lc = dict(synth.layer_cfg(cfg), n_routed=0, top_k=0, n_group=1, topk_group=1)
+    with pytest.raises(qe.ColiError) as ei:
+        qe.router_static(lc, W[:0], b[:0], x, idx=torch.empty((1, 1), dtype=torch.int32, device=DEV),
+                         w=torch.empty((1, 1), device=DEV))
+    assert ei.value.status == qe.COLI_EINVAL
+
+
+def test_router_static_top_p_matches_router():
+    cfg = dict(synth.workload("glm52_decode_int4_t1"), expert_top_p=0.7)
+    W, b = synth.router(cfg, device=DEV)
+    h = _handle(cfg, W, b, max_tokens=8)
+    x = synth.tokens(cfg, T=8, device=DEV, stream=11)
+    idx_ref, w_ref = h.router(x)
+    idx, w = qe.router_static(synth.layer_cfg(cfg), W, b, x)
+    torch.cuda.synchronize()
+    assert (idx_ref < 0).any()
+    np.testing.assert_array_equal(idx.cpu().numpy(), idx_ref.cpu().numpy())
+    np.testing.assert_allclose(w.cpu().numpy(), w_ref.cpu().numpy(), rtol=1e-6)
+    h.close()
