@@ -842,7 +842,7 @@ __device__ __forceinline__ void down_stage_fast_any(int rpw, const uint8_t *stag
 //   P3  gate/up items + SwiGLU + Q8_0(h) records, to global memory; each item
 //       adds one to its expert's count.
 //   P4  experts in the down order (shared first): once an expert's count is
-//       complete, the epilogue warp copies its h records into one of two
+//       complete, the h-fetch warp copies its h records into one of the nh
 //       shared slots and the consumers run its down rows; then the fp64
 //       combine of this CTA's rows, shared experts first.
 struct DecodeArgs {
@@ -1569,6 +1569,9 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
     RingPos rp;
     bool ok = true;
     int n = 0;
+    // one token: the same activation for every item, loaded once
+    LaneAct<BITS, 3> act1;
+    if (MAXT == 1 && geo.fast) act1.load(acts, H, V, fgeo.vbase);
     for (int item = blockIdx.x; item < n_items && ok; item += G, ++n) {
         const int buf = n & 1;
         int a, e, c;
@@ -1578,7 +1581,8 @@ __global__ void __launch_bounds__(DECODE_THREADS, 1) k_moe_decode(DecodeArgs fa)
         const int *tok = lw.pair_tok + p0;
         const bool fast = geo.fast && (MAXT == 1 || ne == 1);
         LaneAct<BITS, 3> act;
-        if (fast) act.load(acts + (size_t)tok[0] * rbH, H, V, fgeo.vbase);
+        if (MAXT == 1) act = act1;
+        else if (fast) act.load(acts + (size_t)tok[0] * rbH, H, V, fgeo.vbase);
         if (n >= 2 && !mbar_wait(&ebars->part_free[buf], (uint32_t)(((n >> 1) - 1) & 1), fa.err, lim)) {
             ok = false;
             *abort = 1;
