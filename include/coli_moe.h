@@ -286,10 +286,10 @@ coli_status coli_dbg_last_forward(coli_moe *m, int T, int32_t *idx, float *w, in
  * COLI_EINVAL.  The fixed array holds 131,328 bytes on every GPU that loads
  * the library, until the process exits.
  * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  Every call on a device shares the one array
- * and it keeps the last call's contents (the ticket is cleared at the start
- * of each call): calls that overlap on the GPU, e.g. on two streams, race. */
+ * (cudaGetSymbolAddress) with that device current.  Every call on a device
+ * shares the one array and it keeps the last call's contents (the ticket is
+ * cleared at the start of each call): calls that overlap on the GPU, e.g. on
+ * two streams, race.  A dense layer (n_routed = 0) returns COLI_EINVAL. */
 coli_status coli_router_static(const coli_moe_config *cfg, const float *router_w,
                                const float *bias, const float *x, int T, int32_t *idx, float *w,
                                coli_stream_t stream);
