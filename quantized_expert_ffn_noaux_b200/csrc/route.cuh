@@ -76,11 +76,12 @@ __global__ void k_route_logits_small(const float *__restrict__ x, int T, int H,
 }
 
 // Logits for many tokens: 64 tokens x 64 experts per CTA, 256 threads each
-// computing a 4 x 4 fp64 tile; K staged through shared memory in fp32.
+// computing a 4 x 4 fp64 tile; K staged through shared memory in fp32, the
+// next 32-wide slice loaded into registers while the current one is used.
 __global__ void __launch_bounds__(256) k_route_logits_tiled(
     const float *__restrict__ x, int T, int H, const float *__restrict__ Wr,
     const float *__restrict__ bias, int E, double *__restrict__ s_out, double *__restrict__ c_out) {
-    constexpr int TM = 64, TN = 64, TK = 32;
+    constexpr int TM = 64, TN = 64, TK = 32, PER = TM * TK / 256;  // 8 values of x and of W per thread
     __shared__ float xs[TK][TM + 1];
     __shared__ float ws[TK][TN + 1];
     const int tid = threadIdx.x;
@@ -91,15 +92,27 @@ __global__ void __launch_bounds__(256) k_route_logits_tiled(
     for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+    // element q of this thread in a slice: row r = (tid + 256 q) / TK, column cc = tid % TK
+    float nx[PER], nw[PER];
+    auto load_slice = [&](int k0) {
+#pragma unroll
+        for (int q = 0; q < PER; ++q) {
+            const int i = tid + 256 * q, r = i / TK, cc = i % TK;
+            const int t = t0 + r, e = e0 + r;
+            nx[q] = (t < T) ? __ldg(x + (int64_t)t * H + k0 + cc) : 0.0f;
+            nw[q] = (e < E) ? __ldg(Wr + (int64_t)e * H + k0 + cc) : 0.0f;
+        }
+    };
+    load_slice(0);
     for (int k0 = 0; k0 < H; k0 += TK) {
-        // 64 rows x 32 cols of x and of W: 2048 floats each, 8 per thread
-        for (int i = tid; i < TM * TK; i += 256) {
-            int r = i / TK, cc = i % TK;
-            int t = t0 + r, e = e0 + r;
-            xs[cc][r] = (t < T) ? __ldg(x + (int64_t)t * H + k0 + cc) : 0.0f;
-            ws[cc][r] = (e < E) ? __ldg(Wr + (int64_t)e * H + k0 + cc) : 0.0f;
+#pragma unroll
+        for (int q = 0; q < PER; ++q) {
+            const int i = tid + 256 * q, r = i / TK, cc = i % TK;
+            xs[cc][r] = nx[q];
+            ws[cc][r] = nw[q];
         }
         __syncthreads();
+        if (k0 + TK < H) load_slice(k0 + TK);  // in flight during this slice's arithmetic
 #pragma unroll 4
         for (int kk = 0; kk < TK; ++kk) {
             double xv[4], wv[4];
