@@ -197,14 +197,16 @@ __global__ void k_gather_pairs(RouteWs ws, const int8_t *__restrict__ xq, const 
 // Per pair, the unsigned-weight offset's share of every row's sum:
 // off * sum_b (sum of the pair's codes in block b) * d_b, in fp64, blocks in
 // order (deterministic).  One CTA per pair; codes [pairs][K] in pair order.
-__global__ void k_pair_offsets(RouteWs ws, const int8_t *__restrict__ q, const float *__restrict__ d, int K,
-                               double off, double *__restrict__ out) {
-    __shared__ double part[256];
+__global__ void __launch_bounds__(256) k_pair_offsets(RouteWs ws, const int8_t *__restrict__ q,
+                                                      const float *__restrict__ d, int K, double off,
+                                                      double *__restrict__ out) {
+    // one warp per pair: lanes stride over the blocks, one fp64 warp sum
     const int np = ws.off[*ws.n_active];
     const int nb = K / COLI_QBLK;
-    for (int p = blockIdx.x; p < np; p += gridDim.x) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int p = (int)blockIdx.x * 8 + warp; p < np; p += (int)gridDim.x * 8) {
         double acc = 0.0;
-        for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+        for (int b = lane; b < nb; b += 32) {
             const int4 *c = reinterpret_cast<const int4 *>(q + (size_t)p * K + (size_t)b * COLI_QBLK);
             const int4 c0 = c[0], c1 = c[1];
             int sx = 0;
@@ -218,14 +220,8 @@ __global__ void k_pair_offsets(RouteWs ws, const int8_t *__restrict__ q, const f
             sx = __dp4a(c1.w, 0x01010101, sx);
             acc = fma((double)sx, (double)d[(size_t)p * nb + b], acc);
         }
-        part[threadIdx.x] = acc;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            double t = 0.0;
-            for (int i = 0; i < (int)blockDim.x; ++i) t += part[i];
-            out[p] = off * t;
-        }
-        __syncthreads();
+        acc = warp_sum(acc);
+        if (lane == 0) out[p] = off * acc;
     }
 }
 
