@@ -711,8 +711,10 @@ coli_status launch_tc_path(coli_moe *m, int T, float *out, cudaStream_t s) {
     st = launch_grouped_tc<BITS>(m, T, 1, s);
     if (st != COLI_OK) return st;
     Launch L(m, s, "combine");
-    k_combine<<<dim3((unsigned)T, (unsigned)((c.hidden + 1023) / 1024)), 256, 0, s>>>(
-        m->rw, m->e_pairs, T, c.hidden, c.top_k, c.n_shared, out, m->out_partial);
+    const int64_t n = (int64_t)T * c.hidden;
+    int grid = (int)std::min<int64_t>((n + 255) / 256, (int64_t)m->nsm * 8);
+    k_combine<<<grid, 256, 0, s>>>(m->rw, m->e_pairs, T, c.hidden, c.top_k, c.n_shared, out,
+                                   m->out_partial);
     return L.done();
 }
 
@@ -768,8 +770,10 @@ coli_status forward_impl(coli_moe *m, const float *x, int T, float *out, cudaStr
         }
         if (st != COLI_OK) return st;
         Launch L(m, s, "combine");
-        k_combine<<<dim3((unsigned)T, (unsigned)((c.hidden + 1023) / 1024)), 256, 0, s>>>(
-            m->rw, m->e_pairs, T, c.hidden, c.top_k, c.n_shared, out, m->out_partial);
+        const int64_t n = (int64_t)T * c.hidden;
+        int grid = (int)std::min<int64_t>((n + 255) / 256, (int64_t)m->nsm * 8);
+        k_combine<<<grid, 256, 0, s>>>(m->rw, m->e_pairs, T, c.hidden, c.top_k, c.n_shared, out,
+                                   m->out_partial);
         st = L.done();
         if (st != COLI_OK) return st;
     }

@@ -256,48 +256,29 @@ __global__ void __launch_bounds__(256) k_down_grouped(RouteWs ws,
 }
 
 // Combine for many tokens: out[t][r] = fp64 sum, shared experts first, then
-// routed slots in order, of weight * e (weight 1 for shared experts).  One
-// CTA per (token, 1024 rows): the token's slot table in shared memory, four
-// consecutive rows per thread (H is a multiple of 32).
-constexpr int COMBINE_MAX_SLOTS = 40;
-__global__ void __launch_bounds__(256) k_combine(RouteWs ws, const float *__restrict__ e_pairs, int T, int H,
-                                                 int k, int S, float *__restrict__ out,
-                                                 double *__restrict__ out_partial) {
-    __shared__ int sp[COMBINE_MAX_SLOTS];
-    __shared__ double sw[COMBINE_MAX_SLOTS];
-    const int t = blockIdx.x, slots = k + S;
-    if ((int)threadIdx.x < slots) {
-        const int jj = threadIdx.x, j = jj < S ? k + jj : jj - S;  // shared experts first
-        sp[jj] = ws.tok_pair[(int64_t)t * slots + j];               // -1: computed by another handle
-        sw[jj] = j < k ? (double)ws.w[(int64_t)t * k + j] : 1.0;
-    }
-    __syncthreads();
-    const int r = 4 * ((int)blockIdx.y * 256 + (int)threadIdx.x);
-    if (r >= H) return;
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int jj = 0; jj < slots; ++jj) {
-        const int p = sp[jj];
-        if (p < 0) continue;
-        const float4 e = *reinterpret_cast<const float4 *>(e_pairs + (int64_t)p * H + r);
-        if (jj < S) {
-            acc[0] += (double)e.x;
-            acc[1] += (double)e.y;
-            acc[2] += (double)e.z;
-            acc[3] += (double)e.w;
-        } else {
-            const double w = sw[jj];
-            acc[0] = fma(w, (double)e.x, acc[0]);
-            acc[1] = fma(w, (double)e.y, acc[1]);
-            acc[2] = fma(w, (double)e.z, acc[2]);
-            acc[3] = fma(w, (double)e.w, acc[3]);
+// routed slots in order, of weight * e (weight 1 for shared experts).
+__global__ void k_combine(RouteWs ws, const float *__restrict__ e_pairs, int T, int H, int k,
+                          int S, float *__restrict__ out, double *__restrict__ out_partial) {
+    const int64_t n = (int64_t)T * H;
+    const int slots = k + S;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int t = (int)(i / H), r = (int)(i % H);
+        double acc = 0.0;
+        for (int jj = 0; jj < slots; ++jj) {
+            const int j = jj < S ? k + jj : jj - S;
+            const int p = ws.tok_pair[(int64_t)t * slots + j];
+            if (p < 0) continue;  // an expert another handle computes
+            const double ev = (double)e_pairs[(int64_t)p * H + r];
+            if (j < k)
+                acc = fma((double)ws.w[(int64_t)t * k + j], ev, acc);
+            else
+                acc += ev;
         }
-    }
-    const int64_t i = (int64_t)t * H + r;
-    if (out_partial) {
-        *reinterpret_cast<double2 *>(out_partial + i) = make_double2(acc[0], acc[1]);
-        *reinterpret_cast<double2 *>(out_partial + i + 2) = make_double2(acc[2], acc[3]);
-    } else {
-        *reinterpret_cast<float4 *>(out + i) = make_float4((float)acc[0], (float)acc[1], (float)acc[2], (float)acc[3]);
+        if (out_partial)
+            out_partial[i] = acc;
+        else
+            out[i] = (float)acc;
     }
 }
 
